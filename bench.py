@@ -1,0 +1,540 @@
+#!/usr/bin/env python3
+"""Benchmark of the W8A8 int8-dynamic linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qkv|ffn_up|ffn_down] [--no-extras] [--no-cpu-baseline]
+
+A step is one whole layer call on one batch: per-token quantization of the
+bf16 activations, the int8 tensor-core GEMM and the fused dequantization
+epilogue (w8a8_linear_fused).  The headline workload is the DiT fused-QKV
+projection, x [4352, 3072] (4096 image + 256 text tokens) against W [9216, 3072].
+Weights are quantized once before timing (load time).  The metric is int8
+TOPS = 2*M*N*K / time of the whole layer (quantization included).
+
+Timing: W warm-up steps, then K steps bracketed by a barrier and a device
+synchronize on both sides, timed with CUDA events on the launching stream;
+the reported time is the max over ranks.  Between steps the inputs rotate
+over several independent buffer sets whose combined size exceeds twice the
+126 MB L2, so no step reads data a previous step left in L2.
+
+Multi-GPU: the layer shards into independent problems, so N ranks run N
+replicas with no collective on the data path (weak scaling); `value` is the
+sum over ranks.  Launched under torchrun, one rank per GPU.
+
+--impl reference times the CPU oracle (plain C, OpenMP) on rank 0 on a
+bounded row sample of the same workload; the other ranks exit without work.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+NOMINAL_INT8_TOPS = 4500.0           # dense int8, B200 datasheet
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+WORKLOADS = {"qkv": synth.QKV, "ffn_up": synth.FFN_UP, "ffn_down": synth.FFN_DOWN}
+
+
+# ----------------------------------------------------------------------------- utils
+
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def bf16_dev(bits: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def n_sets(bytes_per_set: int) -> int:
+    """Buffer sets to rotate so the other sets total more than 2x L2."""
+    return max(3, math.ceil(2 * L2_BYTES / max(bytes_per_set, 1)) + 1)
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.ok = False
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that, do not guess
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def profile_traffic(kernel_tag: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel, or
+    None when the summary is absent or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None, None
+    m = re.search(r"dram_bytes_per_full_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256:\s*([0-9a-f]{16,64})", text)
+    if not m:
+        return None, None
+    if h and h.group(1) != kernel_source_hash()[: len(h.group(1))]:
+        return None, "stale"
+    return float(m.group(1)), "ncu"
+
+
+def kernel_source_hash() -> str:
+    d = os.path.join(ROOT, "w8a8_int8_dynamic_token_b200", "csrc")
+    hs = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, name), "rb") as f:
+                hs.update(f.read())
+    return hs.hexdigest()
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class Layer:
+    """One workload's device buffers, rotated over several independent sets."""
+
+    def __init__(self, case: synth.LayerCase, device, with_ws=True):
+        import w8a8_int8_dynamic_token_b200 as w8a8
+        self.w8a8 = w8a8
+        self.case = case
+        M, K, N = case.M, case.K, case.N
+        x_bits, w_bits, b_bits = case.x(), case.w(), case.b()
+        x0 = bf16_dev(x_bits, device)
+        W = bf16_dev(w_bits, device)
+        Wq, s_w = w8a8.quantize_weights(W)          # load-time weight quantization
+        del W
+        b0 = bf16_dev(b_bits, device) if b_bits is not None else None
+        self.ws_bytes = w8a8.workspace_size(M, N, K) if with_ws else 0
+        per_set = 2 * M * K + N * K + 6 * N + 2 * M * N + self.ws_bytes
+        self.sets = []
+        for _ in range(n_sets(per_set)):
+            self.sets.append({
+                "x": x0.clone(), "Wq": Wq.clone(), "s_w": s_w.clone(),
+                "b": b0.clone() if b0 is not None else None,
+                "y": torch.empty((M, N), dtype=torch.bfloat16, device=device),
+                "ws": torch.empty((max(self.ws_bytes, 16),), dtype=torch.uint8, device=device),
+                "q": torch.empty((M, K), dtype=torch.int8, device=device),
+                "s_a": torch.empty((M,), dtype=torch.float32, device=device),
+            })
+        self.x_host_bits = x_bits
+        self.i = 0
+        self.variant = w8a8.select(M, N, K)["variant_name"]
+        self.launches_per_step = 1 if self.variant == "gemv" else 2
+
+    def step(self):
+        s = self.sets[self.i]
+        self.i = (self.i + 1) % len(self.sets)
+        self.w8a8.linear_fused(s["x"], s["Wq"], s["s_w"], s["b"], out=s["y"], workspace=s["ws"])
+
+    def prepare_gemm_only(self):
+        for s in self.sets:
+            q, s_a = self.w8a8.quant_act(s["x"])
+            s["q"].copy_(q)
+            s["s_a"].copy_(s_a)
+        torch.cuda.synchronize()
+
+    def gemm_step(self):
+        s = self.sets[self.i]
+        self.i = (self.i + 1) % len(self.sets)
+        self.w8a8.linear(s["q"], s["s_a"], s["Wq"], s["s_w"], s["b"], out=s["y"])
+
+    def quant_step(self):
+        s = self.sets[self.i]
+        self.i = (self.i + 1) % len(self.sets)
+        self.w8a8.quant_act(s["x"])
+
+
+def timed(fn, steps: int, warmup: int, dist=None, sampler=None, graph=False):
+    """Run fn warmup times, then time `steps` calls with CUDA events on the
+    current stream, bracketed by barrier + synchronize.  Returns seconds (max
+    over ranks).  graph=True captures the `steps` calls into one CUDA graph
+    first and times its replay (for layers shorter than their host-side
+    launch cost)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(steps):
+                    fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g.replay()                      # one untimed replay
+        torch.cuda.synchronize()
+        fn = g.replay
+        steps_run = 1
+    else:
+        steps_run = steps
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        e0.record(stream)
+        for _ in range(steps_run):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    t = e0.elapsed_time(e1) / 1e3
+    if dist is not None:
+        tt = torch.tensor([t], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+    return t
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def e2e_measure(layer: Layer, steps: int, warmup: int, dist=None):
+    """The same layer through the C ABI call that takes HOST buffers: every
+    step copies x from pinned host memory, runs the layer and copies y back."""
+    w8a8 = layer.w8a8
+    c = layer.case
+    M, K, N = c.M, c.K, c.N
+    dev = torch.device("cuda")
+    x_host = torch.from_numpy(layer.x_host_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    s = layer.sets[0]
+    x_dev = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    y_dev = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+    def fn():
+        w8a8.linear_fused_host(x_host, s["Wq"], s["s_w"], s["b"], y_host, x_dev, y_dev, s["ws"])
+
+    t = timed(fn, steps, warmup, dist)
+    return t, 2 * M * K, 2 * M * N
+
+
+def cpu_baseline(case: synth.LayerCase, budget_s: float = 12.0, max_rows: int = None):
+    """The oracle, as it stands, on a bounded row sample of the workload:
+    quantize the sampled rows, exact int32 GEMM against all N rows of Wq,
+    fp32 epilogue.  Rows are sized from a calibration run to ~budget_s."""
+    import oracle
+    M, K, N = case.M, case.K, case.N
+    x = case.x()
+    wq, sw = oracle.quantize_weights(case.w())
+    b = case.b()
+    rows = 4
+    t0 = time.perf_counter()
+    oracle.linear(x[:rows], wq, sw, b)
+    dt = time.perf_counter() - t0
+    rows = int(max(4, min(M, budget_s / max(dt, 1e-6) * rows)))
+    if max_rows:
+        rows = min(rows, max_rows)
+    t0 = time.perf_counter()
+    oracle.linear(x[:rows], wq, sw, b)
+    dt = time.perf_counter() - t0
+    return {"value": 2.0 * rows * N * K / dt / 1e12, "unit": "TOPS", "cores": oracle.threads(),
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"first {rows} of {M} rows of the {case.name} layer (all {N} outputs per row): "
+                      f"per-token quant + exact int32 GEMM + fp32 epilogue, plain C with OpenMP"}
+
+
+def run_ours(args):
+    rank, world, local = env_rank()
+    dist = None
+    if world > 1:
+        import torch.distributed as tdist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    import w8a8_int8_dynamic_token_b200 as w8a8
+    w8a8.lib()
+    peaks = load_peaks()
+    case = WORKLOADS[args.workload]
+    M, K, N = case.M, case.K, case.N
+    ops = 2.0 * M * N * K
+    warmup = max(3, args.warmup)
+
+    layer = Layer(case, dev)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    t = timed(layer.step, args.steps, warmup, dist, sampler)
+    status = w8a8.last_device_error()
+    if status != 0:
+        raise RuntimeError(f"device error after the timed region: {w8a8.status_string(status)}")
+    sec_per_step = t / args.steps
+    value = world * ops * args.steps / t / 1e12
+
+    # the dominant kernel alone (the tcgen05 GEMM, q precomputed), same rotation
+    layer.prepare_gemm_only()
+    layer.i = 0
+    gsteps = max(args.steps, 50)
+    tg = timed(layer.gemm_step, gsteps, warmup, dist) / gsteps
+    layer.i = 0
+    tq = timed(layer.quant_step, gsteps, warmup, dist) / gsteps
+    int8_peak = peaks["bf16_tflops"] * (NOMINAL_INT8_TOPS / NOMINAL_BF16_TFLOPS)
+    achieved = ops / tg / 1e12
+    traffic, traffic_src = profile_traffic(f"gemm_i8_tcgen05_{case.name}")
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4),
+                "traffic": traffic,
+                "kernel": f"gemm_i8_tcgen05 ({layer.variant})",
+                "peak_basis": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
+                              f"nominal int8/bf16 ratio 2 (int8 ops counted as TOPS)",
+                "frac_of_nominal_4500": round(achieved / NOMINAL_INT8_TOPS, 4),
+                "us_per_launch": round(tg * 1e6, 2)}
+    quant_bytes = 3 * M * K + 4 * M
+    extras = {
+        "layer_us": round(sec_per_step * 1e6, 2),
+        "layer_frac_of_nominal_4500": round(ops / sec_per_step / 1e12 / NOMINAL_INT8_TOPS, 4),
+        "gemm_us": round(tg * 1e6, 2),
+        "quant_us": round(tq * 1e6, 2),
+        "quant_gbs": round(quant_bytes / tq / 1e9, 1),
+        "quant_frac_hbm": round(quant_bytes / tq / 1e9 / peaks["hbm_gbs"], 4),
+    }
+    gpu_launches = layer.launches_per_step * args.steps
+
+    e2e = None
+    if not args.no_e2e:
+        esteps = max(3, min(args.steps, 20))
+        te, h2d, d2h = e2e_measure(layer, esteps, 2, dist)
+        e2e = {"value": round(world * ops * esteps / te / 1e12, 3), "unit": "TOPS",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(te / esteps * 1e3, 3)}
+    del layer
+    torch.cuda.empty_cache()
+
+    components = {}
+    if not args.no_extras:
+        components = extra_components(args, dev, dist, peaks, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(case, budget_s=args.cpu_budget)
+
+    if dist is not None:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": "W8A8 linear int8 TOPS & % of tensor peak (quant+GEMM); M=1 GEMV HBM GB/s",
+            "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": warmup, "ms_per_step": round(sec_per_step * 1e3, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8 (int32 accumulate, fp32 epilogue, bf16 in/out)", "data": "synthetic",
+            "impl": "ours",
+            "config": {"workload": f"{case.name}: x bf16 [{M},{K}] ({case.x_kind}) @ Wq int8 [{N},{K}] + bias -> y bf16",
+                       "M": M, "K": K, "N": N, "seed": case.seed,
+                       "parallelism": f"replicas x{world}",
+                       "l2": f"inputs rotate over independent buffer sets totalling > 2x the 126 MB L2",
+                       "kernel_variant": layer_variant_name(case)},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": gpu_launches,
+            "clocks": sampler.summary(),
+            "extras": extras,
+            "components": components,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def layer_variant_name(case):
+    import w8a8_int8_dynamic_token_b200 as w8a8
+    return w8a8.select(case.M, case.N, case.K)["variant_name"]
+
+
+def extra_components(args, dev, dist, peaks, world):
+    """The other workloads of the same metric: the M = 1 / 2 AdaLN GEMV (HBM
+    GB/s), and the FFN up/down pair, each layer alone and back to back."""
+    out = {}
+    steps = max(20, min(args.steps, 200))
+    for case in (synth.ADALN_M1, synth.ADALN_M2):
+        L = Layer(case, dev)
+        t = timed(L.step, steps * 5, 5, dist, graph=True) / (steps * 5)
+        t_eager = timed(L.step, steps * 5, 5, dist) / (steps * 5)
+        M, K, N = case.M, case.K, case.N
+        algo_bytes = 2 * M * K + N * K + 4 * N + 2 * N + 2 * M * N
+        gbs = algo_bytes / t / 1e9
+        out[case.name] = {"us": round(t * 1e6, 2), "GBs": round(gbs, 1),
+                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                          "TOPS": round(2 * M * N * K / t / 1e12, 3), "variant": L.variant,
+                          "us_eager_launches": round(t_eager * 1e6, 2), "timing": "CUDA graph of back-to-back calls",
+                          "sets_rotated": len(L.sets)}
+        del L
+        torch.cuda.empty_cache()
+    if args.workload == "qkv":
+        layers = {}
+        for case in (synth.FFN_UP, synth.FFN_DOWN):
+            L = Layer(case, dev)
+            t = timed(L.step, steps, 5, dist) / steps
+            ops = 2 * case.M * case.N * case.K
+            out[case.name] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
+                              "frac_of_nominal_4500": round(ops / t / 1e12 / NOMINAL_INT8_TOPS, 4),
+                              "variant": L.variant}
+            layers[case.name] = L
+        up, down = layers["ffn_up"], layers["ffn_down"]
+
+        def pair():
+            up.step()
+            down.step()
+
+        t = timed(pair, steps, 5, dist) / steps
+        ops = 2 * up.case.M * up.case.N * up.case.K + 2 * down.case.M * down.case.N * down.case.K
+        out["ffn_pair"] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
+                           "frac_of_nominal_4500": round(ops / t / 1e12 / NOMINAL_INT8_TOPS, 4)}
+        del layers, up, down
+        torch.cuda.empty_cache()
+    return out
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return
+    import oracle
+    case = WORKLOADS[args.workload]
+    M, K, N = case.M, case.K, case.N
+    x = case.x()
+    wq, sw = oracle.quantize_weights(case.w())
+    b = case.b()
+    # rows per step so the whole run (warmup + steps) takes a few minutes at most
+    t0 = time.perf_counter()
+    oracle.linear(x[:2], wq, sw, b)
+    per_row = (time.perf_counter() - t0) / 2
+    total_steps = max(1, args.steps) + max(3, args.warmup)
+    rows = int(max(1, min(M, 90.0 / total_steps / max(per_row, 1e-9))))
+    for i in range(max(3, args.warmup)):
+        oracle.linear(x[:rows], wq, sw, b)
+    times = []
+    for i in range(max(1, args.steps)):
+        r0 = (i * rows) % max(1, M - rows + 1)
+        t0 = time.perf_counter()
+        oracle.linear(x[r0:r0 + rows], wq, sw, b)
+        times.append(time.perf_counter() - t0)
+    t = sum(times)
+    value = 2.0 * rows * N * K * len(times) / t / 1e12
+    sample = (f"{rows} of {M} rows of the {case.name} layer per step (all {N} outputs per row): "
+              f"per-token quant + exact int32 GEMM + fp32 epilogue, plain C with OpenMP")
+    line = {
+        "metric": "W8A8 linear int8 TOPS & % of tensor peak (quant+GEMM); M=1 GEMV HBM GB/s",
+        "value": round(value, 6), "unit": "TOPS", "n_gpus": world, "steps": len(times),
+        "warmup": max(3, args.warmup), "ms_per_step": round(t / len(times) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8 (int32 accumulate, fp32 epilogue, bf16 in/out)", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": f"{case.name}: x bf16 [{M},{K}] ({case.x_kind}) @ Wq int8 [{N},{K}] + bias -> y bf16",
+                   "M": M, "K": K, "N": N, "seed": case.seed, "parallelism": "rank 0 only"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="qkv")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,201 @@
+/*
+ * w8a8.h -- C ABI of libw8a8.so: the W8A8 int8-dynamic linear layer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (scheme from "Issue 5 probe: int8 quantized DiT serve paths on the
+ * RTX 3090 (24 GB)", section "Round two ... W8A8 int8-dynamic": int8 weights
+ * with fp32 per-output-channel scales, dynamic per-token symmetric int8
+ * activations; "Int8 Quantization" user guide, "Overview" and "Parameters":
+ * activation scales are computed online, static scaling is not supported):
+ *
+ *   s_a[m] = max_k |x[m,k]| / 127                       (fp32, IEEE, RNE)
+ *   q[m,k] = clamp(rint(x[m,k] / s_a[m]), -127, 127)     (ties to even; a row
+ *                                                          with max 0 has s_a = 0, q = 0)
+ *   acc[m,n] = sum_k q[m,k] * Wq[n,k]                   (exact int32)
+ *   y[m,n] = bf16_rne( ((float)acc * s_a[m]) * s_w[n] + (float)bias[n] )
+ *
+ * with Wq, s_w obtained by the same per-row rule from the bf16 weight W[N,K]
+ * (per-output-channel weight quantization: same "Round two" section; "Qwen-Image-2.1:
+ * TE AutoRound-AWQ on GPU + all-resident single-3090 stack", section
+ * "Whole-pipeline follow-up", on per-token activation and per-channel weight
+ * quantization).  The small-M path (M <= 16) serves the AdaLN modulation and
+ * conditioning-embedder layers that run at M = batch (unsloth commit history of
+ * test_diffusion_transformer_quant.py, the commit on torch._int_mm requiring
+ * more than 16 rows).
+ *
+ * Conventions for every call
+ * --------------------------
+ *  - Layouts are row-major.  x bf16 [M,K] (row stride ldx elements), W bf16
+ *    [N,K] (row stride ldw), Wq int8 [N,K] dense (row stride K), q int8 [M,K]
+ *    dense, s_a fp32 [M], s_w fp32 [N], bias bf16 [N] or NULL, y bf16 [M,N]
+ *    (row stride ldy elements).  bf16 values are passed as `const void *` to
+ *    keep this header free of CUDA headers.
+ *  - All tensor pointers are DEVICE pointers owned by the caller, except where
+ *    a call says "host".  The library never allocates memory; scratch memory
+ *    is the caller's `workspace`.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and returns a w8a8_status.  On any error nothing has been
+ *    launched.  Calls never abort the process.
+ *  - Preconditions checked on the host: sizes >= 1; K % 16 == 0 (16-byte int8
+ *    rows for the tensor-memory-accelerator loads); N % 8 == 0 (16-byte bf16
+ *    output rows); K <= 133144 (127*127*K must fit int32); ldx, ldw >= K and
+ *    multiples of 8; ldy >= N and a multiple of 8; every pointer 16-byte
+ *    aligned (s_a 4-byte); the current device is sm_100.
+ *  - Inputs must be finite: NaN or Inf in x or W is outside the contract.
+ *  - Calls on different streams are independent and thread-safe; calls that
+ *    share a workspace must be ordered by the caller.
+ */
+#ifndef W8A8_H
+#define W8A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define W8A8_API __attribute__((visibility("default")))
+#else
+#define W8A8_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *w8a8_stream_t;
+
+typedef enum {
+    W8A8_OK = 0,
+    W8A8_ERR_INVALID_ARG = 1,        /* NULL pointer, size < 1, ld too small */
+    W8A8_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 16, N % 8, K > 133144, ld % 8 */
+    W8A8_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
+    W8A8_ERR_WORKSPACE = 4,          /* workspace NULL or smaller than needed */
+    W8A8_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+    W8A8_ERR_DEVICE_TIMEOUT = 6,     /* a bounded device-side wait gave up */
+    W8A8_ERR_UNSUPPORTED_DEVICE = 7  /* current device is not sm_100 */
+} w8a8_status;
+
+/* Kernel variants, for w8a8_linear_ex / w8a8_select.  AUTO lets the selector
+ * choose from (M, N, K). */
+typedef enum {
+    W8A8_VARIANT_AUTO = 0,
+    W8A8_VARIANT_GEMV = 1,          /* M <= 16: CUDA-core int8 dot products */
+    W8A8_VARIANT_GEMM_BN128 = 2,    /* tcgen05 kind::i8, 128x128 tiles */
+    W8A8_VARIANT_GEMM_BN256 = 3     /* tcgen05 kind::i8, 128x256 tiles */
+} w8a8_variant;
+
+/* The selector's decision for one (M, N, K); see w8a8_select. */
+typedef struct {
+    int32_t variant;       /* a w8a8_variant other than AUTO */
+    int32_t tile_m;        /* rows of y per tile (GEMM) or 0 */
+    int32_t tile_n;        /* columns of y per tile (GEMM) or 0 */
+    int32_t num_tiles;     /* GEMM tiles, or GEMV output rows of W */
+    int32_t grid;          /* CTAs launched */
+    int32_t waves_x100;    /* 100 * num_tiles / grid (GEMM), else 0 */
+} w8a8_plan;
+
+/* Human-readable name of a status code (static string, never NULL). */
+W8A8_API const char *w8a8_status_string(int status);
+
+/*
+ * Weight quantization, run once per layer at load time.
+ * W bf16 [N,K] (row stride ldw) -> Wq int8 [N,K] dense, s_w fp32 [N]:
+ * s_w[n] = max_k |W[n,k]| / 127, Wq = clamp(rint(W / s_w), -127, 127).
+ * Wq is K-major, exactly the layout the GEMM reads (no repacking step).
+ */
+W8A8_API int w8a8_quantize_weights(const void *W_bf16, int64_t N, int64_t K, int64_t ldw,
+                          int8_t *Wq, float *s_w, w8a8_stream_t stream);
+
+/*
+ * Per-token dynamic activation quantization.
+ * x bf16 [M,K] (row stride ldx) -> q int8 [M,K] dense, s_a fp32 [M].
+ */
+W8A8_API int w8a8_quant_act(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
+                   int8_t *q, float *s_a, w8a8_stream_t stream);
+
+/*
+ * Scratch bytes w8a8_linear_fused needs for (M, N, K) (the int8 activations
+ * and their scales when they are not returned through q_out / s_a_out).
+ * w8a8_linear needs none; it accepts workspace = NULL, ws_bytes = 0.
+ */
+W8A8_API int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes);
+
+/*
+ * int8 GEMM + fused epilogue on already-quantized activations.
+ * q int8 [M,K] dense, s_a fp32 [M], Wq int8 [N,K] dense, s_w fp32 [N],
+ * bias bf16 [N] or NULL -> y bf16 [M,N] (row stride ldy).
+ * acc_debug: NULL, or int32 [M,N] dense; when given, the raw int32
+ * accumulators are written there INSTEAD of y (y may then be NULL).
+ * workspace / ws_bytes: unused (may be NULL / 0).
+ */
+W8A8_API int w8a8_linear(const int8_t *q, const float *s_a, int64_t M, int64_t K,
+                const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,
+                void *y_bf16, int64_t ldy, int32_t *acc_debug_or_null,
+                void *workspace, size_t ws_bytes, w8a8_stream_t stream);
+
+/* w8a8_linear with an explicit kernel variant (AUTO = the selector's choice).
+ * GEMV requires M <= 16. */
+W8A8_API int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K,
+                   const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,
+                   void *y_bf16, int64_t ldy, int32_t *acc_debug_or_null,
+                   int variant, w8a8_stream_t stream);
+
+/*
+ * The whole layer from bf16 activations: quantize x per token, then the int8
+ * GEMM with the fused epilogue.  x bf16 [M,K] (row stride ldx) -> y bf16 [M,N].
+ * q_out / s_a_out: NULL, or int8 [M,K] dense / fp32 [M] to receive the
+ * intermediates (then they are used instead of workspace).
+ * workspace: at least w8a8_workspace_size(M,N,K) bytes unless both q_out and
+ * s_a_out are given; 256-byte alignment is recommended.
+ */
+W8A8_API int w8a8_linear_fused(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
+                      const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,
+                      void *y_bf16, int64_t ldy, int8_t *q_out_or_null, float *s_a_out_or_null,
+                      void *workspace, size_t ws_bytes, w8a8_stream_t stream);
+
+/*
+ * End-to-end form of w8a8_linear_fused for callers holding HOST buffers:
+ * enqueues on `stream` the copy x_host -> x_dev, the layer, and the copy
+ * y_dev -> y_host.  x_host: host bf16 [M,K] dense (pinned memory gives
+ * asynchronous copies); y_host: host bf16 [M,N] dense.  x_dev [M,K] dense and
+ * y_dev [M,N] dense are caller-owned device staging buffers; Wq, s_w, bias and
+ * workspace are device pointers as in w8a8_linear_fused.  The call returns
+ * after enqueueing; synchronize `stream` before reading y_host.
+ */
+W8A8_API int w8a8_linear_fused_host(const void *x_host, int64_t M, int64_t K,
+                           const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null,
+                           int64_t N, void *y_host, void *x_dev, void *y_dev,
+                           void *workspace, size_t ws_bytes, w8a8_stream_t stream);
+
+/*
+ * Host-only: the selector's plan for (M, N, K) on a device with num_sms SMs
+ * (148 on B200).  Pure function of its arguments; needs no GPU.
+ */
+W8A8_API int w8a8_select(int64_t M, int64_t N, int64_t K, int32_t num_sms, int variant,
+                w8a8_plan *plan);
+
+/*
+ * Synchronizes `stream`, then reads and clears the library's device error
+ * word.  Returns W8A8_ERR_DEVICE_TIMEOUT if a bounded device-side wait (an
+ * mbarrier wait in a pipelined kernel) gave up since the last call, W8A8_OK
+ * otherwise, or W8A8_ERR_CUDA if the synchronization itself failed.
+ */
+W8A8_API int w8a8_last_device_error(w8a8_stream_t stream);
+
+/*
+ * Self-test of the bounded device-side wait: launches one block that waits,
+ * with a limit of limit_ns nanoseconds (1e3 .. 1e10), on an mbarrier that
+ * nothing ever arrives on.  The wait gives up, records the timeout in the
+ * device error word and the kernel returns; a following
+ * w8a8_last_device_error() reports W8A8_ERR_DEVICE_TIMEOUT.
+ */
+W8A8_API int w8a8_selftest_bounded_wait(int64_t limit_ns, w8a8_stream_t stream);
+
+/* Library version string, e.g. "w8a8 1.0 sm_100a". */
+W8A8_API const char *w8a8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W8A8_H */

@@ -1,0 +1,139 @@
+"""Host-side tests of libw8a8.so that need no GPU: exported symbols, status
+codes, argument checking (which happens before any CUDA call) and the
+selector's decisions."""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import w8a8_int8_dynamic_token_b200 as w8a8
+from w8a8_int8_dynamic_token_b200 import binding as B
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from w8a8_int8_dynamic_token_b200 import build
+    build.build()
+    yield
+
+
+def test_library_exports_every_header_symbol():
+    names = B.header_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(B.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(names) <= exported
+    # only the declared API is exported
+    assert {e for e in exported if e.startswith("w8a8_")} == set(names)
+
+
+def test_binding_covers_every_header_symbol():
+    assert set(B.header_functions()) == set(B._SIGNATURES)
+
+
+def test_status_strings():
+    for st in range(8):
+        assert w8a8.status_string(st) not in ("", "unknown status")
+    assert w8a8.status_string(99) == "unknown status"
+    assert "sm_100a" in w8a8.version()
+
+
+P = ctypes.c_void_p(256)  # never dereferenced: argument errors come first
+
+
+@pytest.mark.parametrize("M,K,ld,expect", [
+    (0, 16, 16, B.W8A8_ERR_INVALID_ARG),
+    (4, 0, 16, B.W8A8_ERR_INVALID_ARG),
+    (4, 32, 16, B.W8A8_ERR_INVALID_ARG),          # ld < K
+    (4, 24, 24, B.W8A8_ERR_UNSUPPORTED_SHAPE),    # K % 16
+    (4, 16, 20, B.W8A8_ERR_UNSUPPORTED_SHAPE),    # ld % 8
+    (4, 133152, 133152, B.W8A8_ERR_UNSUPPORTED_SHAPE),  # K > 133144
+])
+def test_quant_act_argument_errors(M, K, ld, expect):
+    assert B.w8a8_quant_act(P, M, K, ld, P, P, None) == expect
+    assert B.w8a8_quantize_weights(P, M, K, ld, P, P, None) == expect
+
+
+def test_null_and_misaligned_pointers():
+    assert B.w8a8_quant_act(None, 4, 16, 16, P, P, None) == B.W8A8_ERR_INVALID_ARG
+    bad = ctypes.c_void_p(258)
+    assert B.w8a8_quant_act(bad, 4, 16, 16, P, P, None) == B.W8A8_ERR_MISALIGNED
+    assert B.w8a8_linear(P, P, 4, 16, P, P, None, 8, bad, 8, None, None, 0, None) == \
+        B.W8A8_ERR_MISALIGNED
+    assert B.w8a8_linear(P, P, 4, 16, P, P, None, 12, P, 12, None, None, 0, None) == \
+        B.W8A8_ERR_UNSUPPORTED_SHAPE   # N % 8
+    assert B.w8a8_linear_ex(P, P, 4, 16, P, P, None, 8, P, 8, None, 9, None) == \
+        B.W8A8_ERR_INVALID_ARG         # unknown variant
+
+
+def test_valid_arguments_reach_the_device_query():
+    # With valid arguments the call proceeds to the CUDA device query; without
+    # a GPU that reports a CUDA error (on a B200 it would launch).
+    st = B.w8a8_quant_act(P, 4, 16, 16, P, P, None)
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:
+        has_gpu = False
+    if not has_gpu:
+        assert st == B.W8A8_ERR_CUDA
+
+
+def _golden(name):
+    out = {}
+    for line in open(os.path.join(GOLDEN, name)):
+        line = line.split("#", 1)[0].split()
+        if line:
+            out[line[0]] = int(line[1])
+    return out
+
+
+def test_selector_small_m_goes_to_gemv():
+    g = _golden("int_mm_min_rows.txt")
+    lim, K, N = g["int_mm_min_rows_exclusive"], g["adaln_in_features"], g["adaln_out_features"]
+    for M in (1, 2, lim):
+        assert w8a8.select(M, N, K)["variant_name"] == "gemv"
+    assert w8a8.select(lim + 1, N, K)["variant_name"].startswith("gemm")
+    assert w8a8.workspace_size(1, N, K) == 0
+
+
+def test_selector_gemm_plans():
+    p = w8a8.select(4352, 9216, 3072)
+    assert p["variant_name"] == "gemm_bn256" and p["num_tiles"] == 34 * 36 and p["grid"] == 148
+    p = w8a8.select(4352, 3072, 12288)
+    assert p["num_tiles"] == 34 * 12 and p["grid"] == 148
+    # tiny output: few tiles, grid = tiles
+    p = w8a8.select(64, 128, 256)
+    assert p["grid"] == p["num_tiles"] == 1
+    # GEMV would need more than 227 KB of shared memory: falls back to GEMM
+    assert w8a8.select(16, 64, 16384)["variant_name"].startswith("gemm")
+    # forced variants
+    assert w8a8.select(1, 64, 256, variant=B.VARIANT_GEMM_BN128)["tile_n"] == 128
+    with pytest.raises(w8a8.W8A8Error):
+        w8a8.select(17, 64, 256, variant=B.VARIANT_GEMV)
+
+
+def test_workspace_size_covers_q_and_scales():
+    M, N, K = 4352, 9216, 3072
+    n = w8a8.workspace_size(M, N, K)
+    assert n >= M * K + 4 * M and n % 256 == 0
+
+
+@pytest.mark.parametrize("M", [17, 100, 4352, 16384])
+@pytest.mark.parametrize("KN", [(3072, 9216), (3072, 3072), (3072, 12288), (12288, 3072)])
+def test_selector_is_total_and_consistent(M, KN):
+    K, N = KN
+    p = w8a8.select(M, N, K)
+    assert p["variant_name"] in ("gemm_bn128", "gemm_bn256")
+    tn = p["tile_n"]
+    assert p["num_tiles"] == -(-M // 128) * -(-N // tn)
+    assert 1 <= p["grid"] <= 148

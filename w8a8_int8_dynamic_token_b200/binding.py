@@ -1,0 +1,317 @@
+"""ctypes binding of libw8a8.so -- argument marshalling only.
+
+Two layers:
+  * the C-ABI functions under their C names (``w8a8_linear_fused(...)`` etc.),
+    taking raw pointers and sizes exactly as include/w8a8.h declares them;
+  * torch-tensor helpers (``quantize_weights``, ``quant_act``, ``linear``,
+    ``linear_fused``, ...) that check dtypes/devices/strides, allocate outputs
+    with torch, and call the C-ABI on the current CUDA stream.
+
+Every step of the layer runs in the library's CUDA kernels.  There is no CPU
+or PyTorch fallback: if libw8a8.so is missing this module raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libw8a8.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "w8a8.h")
+
+W8A8_OK = 0
+W8A8_ERR_INVALID_ARG = 1
+W8A8_ERR_UNSUPPORTED_SHAPE = 2
+W8A8_ERR_MISALIGNED = 3
+W8A8_ERR_WORKSPACE = 4
+W8A8_ERR_CUDA = 5
+W8A8_ERR_DEVICE_TIMEOUT = 6
+W8A8_ERR_UNSUPPORTED_DEVICE = 7
+
+VARIANT_AUTO = 0
+VARIANT_GEMV = 1
+VARIANT_GEMM_BN128 = 2
+VARIANT_GEMM_BN256 = 3
+VARIANT_NAMES = {0: "auto", 1: "gemv", 2: "gemm_bn128", 3: "gemm_bn256"}
+
+
+class W8A8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("variant", ctypes.c_int32), ("tile_m", ctypes.c_int32),
+                ("tile_n", ctypes.c_int32), ("num_tiles", ctypes.c_int32),
+                ("grid", ctypes.c_int32), ("waves_x100", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+_lib = None
+_vp, _i64, _i32, _int, _sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int,
+                              ctypes.c_size_t)
+
+_SIGNATURES = {
+    "w8a8_status_string": ([_int], ctypes.c_char_p),
+    "w8a8_version": ([], ctypes.c_char_p),
+    "w8a8_quantize_weights": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp], _int),
+    "w8a8_quant_act": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp], _int),
+    "w8a8_workspace_size": ([_i64, _i64, _i64, ctypes.POINTER(_sz)], _int),
+    "w8a8_linear": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp],
+                    _int),
+    "w8a8_linear_ex": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _int, _vp],
+                       _int),
+    "w8a8_linear_fused": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp,
+                           _vp, _sz, _vp], _int),
+    "w8a8_linear_fused_host": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz,
+                                _vp], _int),
+    "w8a8_select": ([_i64, _i64, _i64, _i32, _int, ctypes.POINTER(Plan)], _int),
+    "w8a8_last_device_error": ([_vp], _int),
+    "w8a8_selftest_bounded_wait": ([_i64, _vp], _int),
+}
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/w8a8.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"W8A8_API\s+[^;(]*?\b(w8a8_\w+)\s*\(", text)))
+
+
+def lib() -> ctypes.CDLL:
+    """Load libw8a8.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m w8a8_int8_dynamic_token_b200.build`"
+                " (there is no fallback implementation)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().w8a8_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return lib().w8a8_version().decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != W8A8_OK:
+        raise W8A8Error(status, where)
+
+
+# ------------------------------------------------------------------ raw C ABI
+
+def w8a8_quantize_weights(W, N, K, ldw, Wq, s_w, stream) -> int:
+    return lib().w8a8_quantize_weights(W, N, K, ldw, Wq, s_w, stream)
+
+
+def w8a8_quant_act(x, M, K, ldx, q, s_a, stream) -> int:
+    return lib().w8a8_quant_act(x, M, K, ldx, q, s_a, stream)
+
+
+def w8a8_workspace_size(M, N, K) -> tuple[int, int]:
+    out = ctypes.c_size_t(0)
+    st = lib().w8a8_workspace_size(M, N, K, ctypes.byref(out))
+    return st, int(out.value)
+
+
+def w8a8_linear(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, workspace, ws_bytes,
+                stream) -> int:
+    return lib().w8a8_linear(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, workspace,
+                             ws_bytes, stream)
+
+
+def w8a8_linear_ex(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant, stream) -> int:
+    return lib().w8a8_linear_ex(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant,
+                                stream)
+
+
+def w8a8_linear_fused(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, q_out, s_a_out, workspace,
+                      ws_bytes, stream) -> int:
+    return lib().w8a8_linear_fused(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, q_out, s_a_out,
+                                   workspace, ws_bytes, stream)
+
+
+def w8a8_linear_fused_host(x_host, M, K, Wq, s_w, bias, N, y_host, x_dev, y_dev, workspace,
+                           ws_bytes, stream) -> int:
+    return lib().w8a8_linear_fused_host(x_host, M, K, Wq, s_w, bias, N, y_host, x_dev, y_dev,
+                                        workspace, ws_bytes, stream)
+
+
+def w8a8_select(M, N, K, num_sms=148, variant=VARIANT_AUTO) -> tuple[int, Plan]:
+    plan = Plan()
+    st = lib().w8a8_select(M, N, K, num_sms, variant, ctypes.byref(plan))
+    return st, plan
+
+
+def w8a8_last_device_error(stream) -> int:
+    return lib().w8a8_last_device_error(stream)
+
+
+def w8a8_selftest_bounded_wait(limit_ns, stream) -> int:
+    return lib().w8a8_selftest_bounded_wait(limit_ns, stream)
+
+
+# ------------------------------------------------------------------ torch helpers
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype, ndim, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name} must have unit stride in its last dimension")
+
+
+def workspace_size(M: int, N: int, K: int) -> int:
+    st, n = w8a8_workspace_size(M, N, K)
+    _check(st, "w8a8_workspace_size")
+    return n
+
+
+def select(M: int, N: int, K: int, num_sms: int = 148, variant: int = VARIANT_AUTO) -> dict:
+    st, plan = w8a8_select(M, N, K, num_sms, variant)
+    _check(st, "w8a8_select")
+    d = plan.as_dict()
+    d["variant_name"] = VARIANT_NAMES[d["variant"]]
+    return d
+
+
+def quantize_weights(W: torch.Tensor, stream=None):
+    """bf16 W [N, K] -> (Wq int8 [N, K], s_w fp32 [N]) on W's device."""
+    _need(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    s_w = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _check(w8a8_quantize_weights(_ptr(W), N, K, W.stride(0), _ptr(Wq), _ptr(s_w),
+                                 _stream(stream)), "w8a8_quantize_weights")
+    return Wq, s_w
+
+
+def quant_act(x: torch.Tensor, stream=None):
+    """bf16 x [M, K] -> (q int8 [M, K], s_a fp32 [M])."""
+    _need(x, "x", torch.bfloat16, 2)
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s_a = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check(w8a8_quant_act(_ptr(x), M, K, x.stride(0), _ptr(q), _ptr(s_a), _stream(stream)),
+           "w8a8_quant_act")
+    return q, s_a
+
+
+def linear(q, s_a, Wq, s_w, bias=None, out=None, acc_debug=False, variant=VARIANT_AUTO,
+           stream=None):
+    """y = bf16(((float)(q @ Wq^T) * s_a) * s_w + bias); with acc_debug=True the raw
+    int32 accumulators [M, N] are returned instead."""
+    _need(q, "q", torch.int8, 2)
+    dev = q.device
+    _need(s_a, "s_a", torch.float32, 1, dev)
+    _need(Wq, "Wq", torch.int8, 2, dev)
+    _need(s_w, "s_w", torch.float32, 1, dev)
+    M, K = q.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or s_a.shape[0] != M or s_w.shape[0] != N:
+        raise ValueError("shape mismatch between q, s_a, Wq, s_w")
+    if not (q.is_contiguous() and Wq.is_contiguous()):
+        raise ValueError("q and Wq must be dense row-major")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1, dev)
+        if bias.shape[0] != N:
+            raise ValueError("bias must have N elements")
+    if acc_debug:
+        acc = torch.empty((M, N), dtype=torch.int32, device=dev)
+        _check(w8a8_linear_ex(_ptr(q), _ptr(s_a), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
+                              None, N, _ptr(acc), variant, _stream(stream)), "w8a8_linear_ex")
+        return acc
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(y, "out", torch.bfloat16, 2, dev)
+    _check(w8a8_linear_ex(_ptr(q), _ptr(s_a), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
+                          _ptr(y), y.stride(0), None, variant, _stream(stream)), "w8a8_linear_ex")
+    return y
+
+
+def linear_fused(x, Wq, s_w, bias=None, out=None, workspace=None, return_intermediates=False,
+                 stream=None):
+    """Whole layer from bf16 x [M, K]: per-token quantization, int8 GEMM, fused
+    epilogue.  Returns y [M, N] (and (q, s_a) with return_intermediates=True)."""
+    _need(x, "x", torch.bfloat16, 2)
+    dev = x.device
+    _need(Wq, "Wq", torch.int8, 2, dev)
+    _need(s_w, "s_w", torch.float32, 1, dev)
+    M, K = x.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or s_w.shape[0] != N or not Wq.is_contiguous():
+        raise ValueError("shape mismatch between x, Wq, s_w")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1, dev)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(y, "out", torch.bfloat16, 2, dev)
+    q = s_a = None
+    if return_intermediates:
+        q = torch.empty((M, K), dtype=torch.int8, device=dev)
+        s_a = torch.empty((M,), dtype=torch.float32, device=dev)
+    ws_ptr, ws_bytes = None, 0
+    if not return_intermediates:
+        need = workspace_size(M, N, K)
+        if need:
+            if workspace is None:
+                workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+            if workspace.numel() * workspace.element_size() < need:
+                raise ValueError(f"workspace needs {need} bytes")
+            ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    _check(w8a8_linear_fused(_ptr(x), M, K, x.stride(0), _ptr(Wq), _ptr(s_w), _ptr(bias), N,
+                             _ptr(y), y.stride(0), _ptr(q), _ptr(s_a), ws_ptr, ws_bytes,
+                             _stream(stream)), "w8a8_linear_fused")
+    if return_intermediates:
+        return y, q, s_a
+    return y
+
+
+def linear_fused_host(x_host, Wq, s_w, bias, y_host, x_dev, y_dev, workspace, stream=None):
+    """End-to-end call on host buffers: copy x in, run the layer, copy y out
+    (all enqueued on the stream; synchronize before reading y_host)."""
+    M, K = x_host.shape
+    N = Wq.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(w8a8_linear_fused_host(_ptr(x_host), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
+                                  _ptr(y_host), _ptr(x_dev), _ptr(y_dev), _ptr(workspace),
+                                  ws_bytes, _stream(stream)), "w8a8_linear_fused_host")
+    return y_host
+
+
+def last_device_error(stream=None) -> int:
+    return w8a8_last_device_error(_stream(stream))
+
+
+def selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    return w8a8_selftest_bounded_wait(int(limit_ns), _stream(stream))

@@ -1,0 +1,540 @@
+// w8a8_capi.cu -- the C ABI of libw8a8.so (declared in include/w8a8.h):
+// argument checks, the (M, N, K) -> kernel selector, TMA descriptor encoding
+// and kernel launches.  The library allocates no memory; all scratch memory
+// is the caller's workspace.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/w8a8.h"
+#include "w8a8_gemm.cuh"
+#include "w8a8_gemv.cuh"
+#include "w8a8_ptx.cuh"
+#include "w8a8_quant.cuh"
+
+namespace w8a8 {
+
+constexpr int64_t kMaxK = 133144;  // 127 * 127 * K <= 2^31 - 1
+constexpr int kMaxDevices = 64;
+constexpr int kGemmStages256 = 4;  // 4 x 48 KB ring for 128x256 tiles
+constexpr int kGemmStages128 = 6;  // 6 x 32 KB ring for 128x128 tiles
+constexpr int kGemmGroupM = 8;
+
+// ---------------------------------------------------------------- device info
+
+struct DeviceInfo {
+  std::atomic<int> state{0};  // 0 unknown, 1 ready
+  int cc_major = 0, cc_minor = 0, sms = 0, max_smem_optin = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+int query_device(const DeviceInfo **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  DeviceInfo &d = g_dev[dev];
+  if (d.state.load(std::memory_order_acquire) != 1) {
+    int maj = 0, min = 0, sms = 0, smem = 0;
+    if (cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&min, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess) {
+      cudaGetLastError();
+      return W8A8_ERR_CUDA;
+    }
+    d.cc_major = maj;
+    d.cc_minor = min;
+    d.sms = sms;
+    d.max_smem_optin = smem;
+    d.state.store(1, std::memory_order_release);
+  }
+  if (d.cc_major != 10 || d.cc_minor != 0) return W8A8_ERR_UNSUPPORTED_DEVICE;
+  *out = &d;
+  return W8A8_OK;
+}
+
+// ---------------------------------------------------------------- checks
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_mk(int64_t M, int64_t K, int64_t ld) {
+  if (M < 1 || K < 1 || ld < K) return W8A8_ERR_INVALID_ARG;
+  if (K % 16 != 0 || K > kMaxK || ld % 8 != 0) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  if (M > INT32_MAX / 2) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  return W8A8_OK;
+}
+
+int check_n(int64_t N, int64_t ldy) {
+  if (N < 1 || ldy < N) return W8A8_ERR_INVALID_ARG;
+  if (N % 8 != 0 || ldy % 8 != 0 || N > INT32_MAX / 2) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  return W8A8_OK;
+}
+
+// ---------------------------------------------------------------- selector
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline bool gemv_fits(int64_t M, int64_t K, int max_smem) {
+  return M <= kGemvMaxM && M * K + 1024 <= static_cast<int64_t>(max_smem);
+}
+
+int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int max_smem,
+                w8a8_plan *plan) {
+  if (sms < 1) return W8A8_ERR_INVALID_ARG;
+  int v = variant;
+  if (v == W8A8_VARIANT_AUTO) {
+    if (gemv_fits(M, K, max_smem)) {
+      v = W8A8_VARIANT_GEMV;
+    } else {
+      // wave efficiency of each tile width; 256-wide tiles move half the
+      // activation bytes per op, so 128-wide tiles must win clearly
+      const int64_t t256 = cdiv(M, kBM) * cdiv(N, 256);
+      const int64_t t128 = cdiv(M, kBM) * cdiv(N, 128);
+      const double e256 = static_cast<double>(t256) / (cdiv(t256, sms) * sms) *
+                          (static_cast<double>(N) / (cdiv(N, 256) * 256));
+      const double e128 = static_cast<double>(t128) / (cdiv(t128, sms) * sms) *
+                          (static_cast<double>(N) / (cdiv(N, 128) * 128));
+      v = (e128 > 1.15 * e256) ? W8A8_VARIANT_GEMM_BN128 : W8A8_VARIANT_GEMM_BN256;
+    }
+  }
+  std::memset(plan, 0, sizeof(*plan));
+  plan->variant = v;
+  if (v == W8A8_VARIANT_GEMV) {
+    if (!gemv_fits(M, K, max_smem)) return W8A8_ERR_UNSUPPORTED_SHAPE;
+    const int64_t smem = M * K;
+    int per_sm = static_cast<int>((max_smem) / (smem + 1024));
+    per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+    const int64_t rows_per_cta = kGemvThreads / 32;
+    int64_t grid = cdiv(N, rows_per_cta);
+    const int64_t cap = static_cast<int64_t>(sms) * per_sm;
+    plan->num_tiles = static_cast<int32_t>(N);
+    plan->grid = static_cast<int32_t>(grid < cap ? grid : cap);
+    return W8A8_OK;
+  }
+  if (v != W8A8_VARIANT_GEMM_BN128 && v != W8A8_VARIANT_GEMM_BN256) return W8A8_ERR_INVALID_ARG;
+  const int bn = v == W8A8_VARIANT_GEMM_BN128 ? 128 : 256;
+  const int64_t tiles = cdiv(M, kBM) * cdiv(N, bn);
+  if (tiles > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  plan->tile_m = kBM;
+  plan->tile_n = bn;
+  plan->num_tiles = static_cast<int32_t>(tiles);
+  plan->grid = static_cast<int32_t>(tiles < sms ? tiles : sms);
+  plan->waves_x100 = static_cast<int32_t>(100 * tiles / plan->grid);
+  return W8A8_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  PFN_cuTensorMapEncodeTiled_v12000 f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    fn.store(f, std::memory_order_release);
+  }
+  return f;
+}
+
+// int8 matrix [rows, K] dense, box = 128 (K) x box_rows, 128-byte swizzle.
+int encode_i8_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return W8A8_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- launches
+
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+           Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  return W8A8_OK;
+}
+
+template <typename K>
+int set_smem_attr(K kernel, int bytes) {
+  if (cudaFuncSetAttribute(reinterpret_cast<const void *>(kernel),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  return W8A8_OK;
+}
+
+int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q, float *s,
+                 cudaStream_t stream) {
+  const int64_t nvec = K / 8;
+  int G = 32;
+  int64_t V = cdiv(nvec, G);
+  while (V > 8 && G < 1024) {
+    G *= 2;
+    V = cdiv(nvec, G);
+  }
+  const int block = G > 256 ? G : 256;
+  const int rows_per_block = block / G;
+  const int64_t grid = cdiv(rows, rows_per_block);
+  if (grid > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  const uint16_t *xp = static_cast<const uint16_t *>(x);
+#define W8A8_QUANT_CASE(VV)                                                                   \
+  return launch(quant_rows_kernel<VV>, dim3(static_cast<unsigned>(grid)), dim3(block), 0,     \
+                stream, xp, rows, K, ldx, q, s, G)
+  switch (V) {
+    case 1: W8A8_QUANT_CASE(1);
+    case 2: W8A8_QUANT_CASE(2);
+    case 3: W8A8_QUANT_CASE(3);
+    case 4: W8A8_QUANT_CASE(4);
+    case 5: W8A8_QUANT_CASE(5);
+    case 6: W8A8_QUANT_CASE(6);
+    case 7: W8A8_QUANT_CASE(7);
+    case 8: W8A8_QUANT_CASE(8);
+    case 9: case 10: case 11: case 12: W8A8_QUANT_CASE(12);
+    default: W8A8_QUANT_CASE(17);  // G = 1024, K <= 133144 -> V <= 17
+  }
+#undef W8A8_QUANT_CASE
+}
+
+template <int BN, int STAGES, bool RAW>
+int launch_gemm_t(const w8a8_plan &plan, const int8_t *q, const float *s_a, int64_t M,
+                  int64_t K, const int8_t *wq, const float *s_w, const void *bias, int64_t N,
+                  void *y, int64_t ldy, int32_t *acc, cudaStream_t stream) {
+  using L = GemmLayout<BN, STAGES>;
+  CUtensorMap ma, mb;
+  int st = encode_i8_map(&ma, q, M, K, kBM);
+  if (st != W8A8_OK) return st;
+  st = encode_i8_map(&mb, wq, N, K, BN);
+  if (st != W8A8_OK) return st;
+  GemmParams p;
+  p.M = static_cast<int32_t>(M);
+  p.N = static_cast<int32_t>(N);
+  p.K = static_cast<int32_t>(K);
+  p.num_m_blk = static_cast<int32_t>(cdiv(M, kBM));
+  p.num_n_blk = static_cast<int32_t>(cdiv(N, BN));
+  p.num_tiles = plan.num_tiles;
+  p.k_blocks = static_cast<int32_t>(cdiv(K, kBK));
+  p.group_m = kGemmGroupM;
+  p.s_a = s_a;
+  p.s_w = s_w;
+  p.bias = static_cast<const uint16_t *>(bias);
+  p.y = static_cast<uint16_t *>(y);
+  p.ldy = ldy;
+  p.acc_out = acc;
+  auto kernel = gemm_i8_tcgen05_kernel<BN, STAGES, RAW>;
+  st = set_smem_attr(kernel, L::kSmemBytes);
+  if (st != W8A8_OK) return st;
+  return launch(kernel, dim3(plan.grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma, mb, p);
+}
+
+template <bool FUSED, bool RAW>
+int launch_gemv_m(const w8a8_plan &plan, const GemvParams &p, int max_smem,
+                  cudaStream_t stream) {
+  const int smem = p.M * p.K;
+  (void)max_smem;
+#define W8A8_GEMV_CASE(MT)                                                              \
+  {                                                                                     \
+    auto kernel = gemv_i8_kernel<MT, FUSED, RAW>;                                       \
+    int st = set_smem_attr(kernel, smem);                                               \
+    if (st != W8A8_OK) return st;                                                       \
+    return launch(kernel, dim3(plan.grid), dim3(kGemvThreads), smem, stream, p);        \
+  }
+  if (p.M <= 1) W8A8_GEMV_CASE(1)
+  if (p.M <= 2) W8A8_GEMV_CASE(2)
+  if (p.M <= 4) W8A8_GEMV_CASE(4)
+  if (p.M <= 8) W8A8_GEMV_CASE(8)
+  W8A8_GEMV_CASE(16)
+#undef W8A8_GEMV_CASE
+}
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+size_t fused_workspace_bytes(int64_t M, int64_t K) {
+  return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
+         align256(static_cast<size_t>(M) * sizeof(float));
+}
+
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the wait must give up after limit_ns
+  if (threadIdx.x == 0) mbar_wait(&bar, 0u, &abort_flag, limit_ns);
+}
+
+int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
+                const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
+                int32_t *acc, int variant, cudaStream_t stream) {
+  if (!q || !s_a || !Wq || !s_w || (!y && !acc)) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(M, K, K);
+  if (st != W8A8_OK) return st;
+  st = check_n(N, acc ? (ldy >= N ? ldy : N) : ldy);
+  if (st != W8A8_OK) return st;
+  if (!aligned16(q) || !aligned16(Wq) || !aligned16(s_w) || (bias && !aligned16(bias)) ||
+      (y && !aligned16(y)) || (acc && !aligned16(acc)) ||
+      (reinterpret_cast<uintptr_t>(s_a) & 3u))
+    return W8A8_ERR_MISALIGNED;
+  const DeviceInfo *d = nullptr;
+  st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  w8a8_plan plan;
+  st = select_plan(M, N, K, d->sms, variant, d->max_smem_optin, &plan);
+  if (st != W8A8_OK) return st;
+  if (plan.variant == W8A8_VARIANT_GEMV) {
+    GemvParams p = {};
+    p.M = static_cast<int32_t>(M);
+    p.N = static_cast<int32_t>(N);
+    p.K = static_cast<int32_t>(K);
+    p.q = q;
+    p.s_a = s_a;
+    p.wq = Wq;
+    p.s_w = s_w;
+    p.bias = static_cast<const uint16_t *>(bias);
+    p.y = static_cast<uint16_t *>(y);
+    p.ldy = ldy;
+    p.acc_out = acc;
+    return acc ? launch_gemv_m<false, true>(plan, p, d->max_smem_optin, stream)
+               : launch_gemv_m<false, false>(plan, p, d->max_smem_optin, stream);
+  }
+  if (plan.variant == W8A8_VARIANT_GEMM_BN128) {
+    return acc ? launch_gemm_t<128, kGemmStages128, true>(plan, q, s_a, M, K, Wq, s_w, bias, N,
+                                                           y, ldy, acc, stream)
+               : launch_gemm_t<128, kGemmStages128, false>(plan, q, s_a, M, K, Wq, s_w, bias,
+                                                            N, y, ldy, acc, stream);
+  }
+  return acc ? launch_gemm_t<256, kGemmStages256, true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y,
+                                                         ldy, acc, stream)
+             : launch_gemm_t<256, kGemmStages256, false>(plan, q, s_a, M, K, Wq, s_w, bias, N,
+                                                          y, ldy, acc, stream);
+}
+
+}  // namespace w8a8
+
+using namespace w8a8;
+
+extern "C" {
+
+const char *w8a8_status_string(int status) {
+  switch (status) {
+    case W8A8_OK: return "ok";
+    case W8A8_ERR_INVALID_ARG: return "invalid argument (null pointer, size < 1 or stride too small)";
+    case W8A8_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (need K % 16 == 0, N % 8 == 0, K <= 133144, strides % 8 == 0)";
+    case W8A8_ERR_MISALIGNED: return "misaligned pointer (16-byte alignment required)";
+    case W8A8_ERR_WORKSPACE: return "workspace missing or too small";
+    case W8A8_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case W8A8_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+    case W8A8_ERR_UNSUPPORTED_DEVICE: return "unsupported device (sm_100 required)";
+    default: return "unknown status";
+  }
+}
+
+const char *w8a8_version(void) { return "w8a8 1.0 sm_100a"; }
+
+int w8a8_quantize_weights(const void *W, int64_t N, int64_t K, int64_t ldw, int8_t *Wq,
+                          float *s_w, w8a8_stream_t stream) {
+  if (!W || !Wq || !s_w) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(N, K, ldw);
+  if (st != W8A8_OK) return st;
+  if (!aligned16(W) || !aligned16(Wq) || (reinterpret_cast<uintptr_t>(s_w) & 3u))
+    return W8A8_ERR_MISALIGNED;
+  const DeviceInfo *d = nullptr;
+  st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  return launch_quant(W, N, K, ldw, Wq, s_w, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8a8_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q, float *s_a,
+                   w8a8_stream_t stream) {
+  if (!x || !q || !s_a) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(M, K, ldx);
+  if (st != W8A8_OK) return st;
+  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s_a) & 3u))
+    return W8A8_ERR_MISALIGNED;
+  const DeviceInfo *d = nullptr;
+  st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  return launch_quant(x, M, K, ldx, q, s_a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8a8_select(int64_t M, int64_t N, int64_t K, int32_t num_sms, int variant,
+                w8a8_plan *plan) {
+  if (!plan) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(M, K, K);
+  if (st != W8A8_OK) return st;
+  st = check_n(N, N);
+  if (st != W8A8_OK) return st;
+  // B200: 227 KB of opt-in shared memory per block
+  return select_plan(M, N, K, num_sms, variant, 232448, plan);
+}
+
+int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes) {
+  if (!bytes) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(M, K, K);
+  if (st != W8A8_OK) return st;
+  st = check_n(N, N);
+  if (st != W8A8_OK) return st;
+  w8a8_plan plan;
+  st = select_plan(M, N, K, 148, W8A8_VARIANT_AUTO, 232448, &plan);
+  if (st != W8A8_OK) return st;
+  *bytes = plan.variant == W8A8_VARIANT_GEMV ? 0 : fused_workspace_bytes(M, K);
+  return W8A8_OK;
+}
+
+int w8a8_linear(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
+                const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
+                int32_t *acc_debug, void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, W8A8_VARIANT_AUTO,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
+                   const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
+                   int32_t *acc_debug, int variant, w8a8_stream_t stream) {
+  if (variant < W8A8_VARIANT_AUTO || variant > W8A8_VARIANT_GEMM_BN256)
+    return W8A8_ERR_INVALID_ARG;
+  return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t *Wq,
+                      const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
+                      int8_t *q_out, float *s_a_out, void *workspace, size_t ws_bytes,
+                      w8a8_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!x || !Wq || !s_w || !y) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(M, K, ldx);
+  if (st != W8A8_OK) return st;
+  st = check_n(N, ldy);
+  if (st != W8A8_OK) return st;
+  if (!aligned16(x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(y) ||
+      (bias && !aligned16(bias)) || (q_out && !aligned16(q_out)) ||
+      (s_a_out && (reinterpret_cast<uintptr_t>(s_a_out) & 3u)))
+    return W8A8_ERR_MISALIGNED;
+  const DeviceInfo *d = nullptr;
+  st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  w8a8_plan plan;
+  st = select_plan(M, N, K, d->sms, W8A8_VARIANT_AUTO, d->max_smem_optin, &plan);
+  if (st != W8A8_OK) return st;
+
+  if (plan.variant == W8A8_VARIANT_GEMV) {
+    GemvParams p = {};
+    p.M = static_cast<int32_t>(M);
+    p.N = static_cast<int32_t>(N);
+    p.K = static_cast<int32_t>(K);
+    p.x = static_cast<const uint16_t *>(x);
+    p.ldx = ldx;
+    p.wq = Wq;
+    p.s_w = s_w;
+    p.bias = static_cast<const uint16_t *>(bias);
+    p.y = static_cast<uint16_t *>(y);
+    p.ldy = ldy;
+    p.q_out = q_out;
+    p.s_a_out = s_a_out;
+    return launch_gemv_m<true, false>(plan, p, d->max_smem_optin, stream);
+  }
+
+  int8_t *q = q_out;
+  float *s_a = s_a_out;
+  if (!q || !s_a) {
+    const size_t need = fused_workspace_bytes(M, K);
+    if (!workspace || ws_bytes < need || !aligned16(workspace)) return W8A8_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (!q) q = reinterpret_cast<int8_t *>(ws);
+    if (!s_a) s_a = reinterpret_cast<float *>(ws + align256(static_cast<size_t>(M * K)));
+  }
+  st = launch_quant(x, M, K, ldx, q, s_a, stream);
+  if (st != W8A8_OK) return st;
+  return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, nullptr, plan.variant, stream);
+}
+
+int w8a8_linear_fused_host(const void *x_host, int64_t M, int64_t K, const int8_t *Wq,
+                           const float *s_w, const void *bias, int64_t N, void *y_host,
+                           void *x_dev, void *y_dev, void *workspace, size_t ws_bytes,
+                           w8a8_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!x_host || !y_host || !x_dev || !y_dev) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(M, K, K);
+  if (st != W8A8_OK) return st;
+  st = check_n(N, N);
+  if (st != W8A8_OK) return st;
+  const DeviceInfo *d = nullptr;
+  st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  if (cudaMemcpyAsync(x_dev, x_host, static_cast<size_t>(M * K) * 2, cudaMemcpyHostToDevice,
+                      stream) != cudaSuccess) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  st = w8a8_linear_fused(x_dev, M, K, K, Wq, s_w, bias, N, y_dev, N, nullptr, nullptr, workspace,
+                         ws_bytes, stream_);
+  if (st != W8A8_OK) return st;
+  if (cudaMemcpyAsync(y_host, y_dev, static_cast<size_t>(M * N) * 2, cudaMemcpyDeviceToHost,
+                      stream) != cudaSuccess) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  return W8A8_OK;
+}
+
+int w8a8_last_device_error(w8a8_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  return (word & W8A8_DEVERR_TIMEOUT) ? W8A8_ERR_DEVICE_TIMEOUT : W8A8_OK;
+}
+
+int w8a8_selftest_bounded_wait(int64_t limit_ns, w8a8_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000LL) return W8A8_ERR_INVALID_ARG;
+  const DeviceInfo *d = nullptr;
+  int st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  return launch(bounded_wait_selftest_kernel, dim3(1), dim3(32), 0,
+                reinterpret_cast<cudaStream_t>(stream), static_cast<uint64_t>(limit_ns));
+}
+
+}  // extern "C"

@@ -1,0 +1,168 @@
+// w8a8_gemv.cuh -- the W8A8 layer for M <= 16 activation rows.
+//
+// At M = batch (1, or 2 under classifier-free guidance) the AdaLN modulation
+// and conditioning-embedder linears are matrix-vector products (unsloth commit
+// history of test_diffusion_transformer_quant.py: the commit on torch._int_mm
+// needing more than 16 rows, e.g. Flux norm1.linear 3072 -> 18432 at M = 1).
+// Their cost is streaming the int8 weight matrix from HBM once, so this kernel
+// is built around that stream:
+//   1. (fused variant) every CTA quantizes the M activation rows into shared
+//      memory with the per-token rule of the quantization kernel;
+//      (unfused variant) every CTA copies the given q rows into shared memory;
+//   2. each warp walks whole weight rows n, lanes reading 16-byte vectors with
+//      evict-first loads, accumulating M int32 dot products with dp4a
+//      (exact: every partial sum is bounded by 127*127*K < 2^31);
+//   3. a warp reduction, then lane m writes
+//      y[m,n] = bf16_rne(((float)acc * s_a[m]) * s_w[n] + (float)bias[n]).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "w8a8_quant.cuh"
+
+namespace w8a8 {
+
+constexpr int kGemvThreads = 256;
+constexpr int kGemvMaxM = 16;
+
+struct GemvParams {
+  int32_t M, N, K;
+  const uint16_t *x;  // bf16 [M, K], row stride ldx (fused variant)
+  int64_t ldx;
+  const int8_t *q;    // int8 [M, K] dense (unfused variant)
+  const float *s_a;   // [M] (unfused variant)
+  const int8_t *wq;   // [N, K] dense
+  const float *s_w;
+  const uint16_t *bias;  // or nullptr
+  uint16_t *y;
+  int64_t ldy;
+  int32_t *acc_out;   // raw int32 [M, N] dense instead of y (debug), or nullptr
+  int8_t *q_out;      // fused variant: optional copy of q (written by CTA 0)
+  float *s_a_out;     // fused variant: optional copy of s_a
+};
+
+// Block-wide max of non-negative 16-bit patterns.
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();  // red[] may still be read from the previous call
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = 0u;
+#pragma unroll
+  for (int w = 0; w < kGemvThreads / 32; ++w) v = max(v, red[w]);
+  return v;
+}
+
+template <int MT, bool FUSED, bool RAW_OUT>
+__global__ void __launch_bounds__(kGemvThreads) gemv_i8_kernel(const GemvParams p) {
+  extern __shared__ __align__(16) uint8_t gemv_smem[];
+  int8_t *qs = reinterpret_cast<int8_t *>(gemv_smem);  // [M][K]
+  __shared__ float sas[kGemvMaxM];
+  __shared__ uint32_t red[kGemvThreads / 32];
+
+  const int tid = threadIdx.x;
+  const int K = p.K;
+  const int nvec8 = K >> 3;    // 8-element bf16 vectors per row
+  const int nvec16 = K >> 4;   // 16-byte int8 vectors per row
+
+  // ---- 1. activation rows -> shared memory (int8) + scales
+  if constexpr (FUSED) {
+    for (int m = 0; m < p.M; ++m) {
+      const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(m) * p.ldx);
+      uint32_t mm = 0u;
+      for (int v = tid; v < nvec8; v += kGemvThreads) {
+        const uint4 a = __ldg(xr + v);
+        mm = bf16x2_absmax(mm, a.x);
+        mm = bf16x2_absmax(mm, a.y);
+        mm = bf16x2_absmax(mm, a.z);
+        mm = bf16x2_absmax(mm, a.w);
+      }
+      const uint32_t mb = block_max_u32(bf16x2_max_halves(mm), red);
+      const float amax = __uint_as_float(mb << 16);
+      const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+      if (tid == 0) sas[m] = sc;
+      uint2 *qrow = reinterpret_cast<uint2 *>(qs + m * K);
+      for (int v = tid; v < nvec8; v += kGemvThreads) {
+        const uint4 a = __ldg(xr + v);
+        qrow[v] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(a, sc);
+      }
+    }
+  } else {
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.q);
+    uint4 *dst = reinterpret_cast<uint4 *>(qs);
+    for (int v = tid; v < p.M * nvec16; v += kGemvThreads) dst[v] = __ldg(src + v);
+    if (tid < p.M) sas[tid] = __ldg(p.s_a + tid);
+  }
+  __syncthreads();
+  if constexpr (FUSED) {
+    if (blockIdx.x == 0) {
+      if (p.q_out != nullptr) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(qs);
+        uint4 *dst = reinterpret_cast<uint4 *>(p.q_out);
+        for (int v = tid; v < p.M * nvec16; v += kGemvThreads) dst[v] = src[v];
+      }
+      if (p.s_a_out != nullptr && tid < p.M) p.s_a_out[tid] = sas[tid];
+    }
+  }
+
+  // ---- 2. stream weight rows
+  const int warp = tid >> 5, lane = tid & 31;
+  const int warps_total = gridDim.x * (kGemvThreads / 32);
+  constexpr int U = 4;  // 16-byte weight vectors in flight per lane
+  for (int n = blockIdx.x * (kGemvThreads / 32) + warp; n < p.N; n += warps_total) {
+    const uint4 *wr = reinterpret_cast<const uint4 *>(p.wq + static_cast<int64_t>(n) * K);
+    int acc[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[m] = 0;
+    for (int base = lane; base < nvec16; base += 32 * U) {
+      uint4 wv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int vi = base + 32 * u;
+        wv[u] = vi < nvec16 ? __ldcs(wr + vi) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int vi = base + 32 * u;
+        if (vi < nvec16) {
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            if (m < p.M) {
+              const int4 qv = reinterpret_cast<const int4 *>(qs + m * K)[vi];
+              acc[m] = __dp4a(static_cast<int>(wv[u].x), qv.x, acc[m]);
+              acc[m] = __dp4a(static_cast<int>(wv[u].y), qv.y, acc[m]);
+              acc[m] = __dp4a(static_cast<int>(wv[u].z), qv.z, acc[m]);
+              acc[m] = __dp4a(static_cast<int>(wv[u].w), qv.w, acc[m]);
+            }
+          }
+        }
+      }
+    }
+    // ---- 3. reduce across the warp, lane m finishes row m
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[m] += __shfl_xor_sync(0xFFFFFFFFu, acc[m], o);
+    }
+    int mine = 0;
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+      if (lane == m) mine = acc[m];
+    if (lane < p.M) {
+      if constexpr (RAW_OUT) {
+        p.acc_out[static_cast<int64_t>(lane) * p.N + n] = mine;
+      } else {
+        float v = __int2float_rn(mine);
+        v = __fmul_rn(__fmul_rn(v, sas[lane]), __ldg(p.s_w + n));
+        if (p.bias != nullptr) v = __fadd_rn(v, __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16));
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        p.y[static_cast<int64_t>(lane) * p.ldy + n] = *reinterpret_cast<const uint16_t *>(&h);
+      }
+    }
+  }
+}
+
+}  // namespace w8a8
