@@ -196,18 +196,24 @@ int set_smem_attr(K kernel, int bytes) {
 
 int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q, float *s,
                  cudaStream_t stream) {
+  // G threads per row (32..256) holding V <= 8 vectors of 8 bf16 each in
+  // registers; longer rows take the two-pass kernel.
   const int64_t nvec = K / 8;
   int G = 32;
   int64_t V = cdiv(nvec, G);
-  while (V > 8 && G < 1024) {
+  while (V > 8 && G < 256) {
     G *= 2;
     V = cdiv(nvec, G);
   }
-  const int block = G > 256 ? G : 256;
+  const uint16_t *xp = static_cast<const uint16_t *>(x);
+  if (rows > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  if (V > 8) {
+    return launch(quant_rows_long_kernel, dim3(static_cast<unsigned>(rows)), dim3(256), 0, stream,
+                  xp, K, ldx, q, s);
+  }
+  const int block = 256;
   const int rows_per_block = block / G;
   const int64_t grid = cdiv(rows, rows_per_block);
-  if (grid > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
-  const uint16_t *xp = static_cast<const uint16_t *>(x);
 #define W8A8_QUANT_CASE(VV)                                                                   \
   return launch(quant_rows_kernel<VV>, dim3(static_cast<unsigned>(grid)), dim3(block), 0,     \
                 stream, xp, rows, K, ldx, q, s, G)
@@ -219,9 +225,7 @@ int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q,
     case 5: W8A8_QUANT_CASE(5);
     case 6: W8A8_QUANT_CASE(6);
     case 7: W8A8_QUANT_CASE(7);
-    case 8: W8A8_QUANT_CASE(8);
-    case 9: case 10: case 11: case 12: W8A8_QUANT_CASE(12);
-    default: W8A8_QUANT_CASE(17);  // G = 1024, K <= 133144 -> V <= 17
+    default: W8A8_QUANT_CASE(8);
   }
 #undef W8A8_QUANT_CASE
 }

@@ -128,4 +128,42 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t *__restr
   }
 }
 
+// Long rows (more than 256 threads x 8 vectors): one block of 256 threads per
+// row, two passes over the row -- max |x| first, then quantize -- the second
+// pass reading the row back from L2.
+__global__ void __launch_bounds__(256) quant_rows_long_kernel(const uint16_t *__restrict__ x,
+                                                              int64_t K, int64_t ldx,
+                                                              int8_t *__restrict__ q,
+                                                              float *__restrict__ s) {
+  __shared__ uint32_t red[8];
+  const int64_t row = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int64_t nvec = K >> 3;
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * ldx);
+  uint32_t m = 0u;
+  for (int64_t vi = tid; vi < nvec; vi += 256) {
+    const uint4 v = __ldg(xr + vi);
+    m = bf16x2_absmax(m, v.x);
+    m = bf16x2_absmax(m, v.y);
+    m = bf16x2_absmax(m, v.z);
+    m = bf16x2_absmax(m, v.w);
+  }
+  uint32_t mb = bf16x2_max_halves(m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mb;
+  __syncthreads();
+  mb = 0u;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) mb = max(mb, red[w]);
+  const float amax = __uint_as_float(mb << 16);
+  const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+  if (tid == 0) s[row] = sc;
+  uint2 *qr = reinterpret_cast<uint2 *>(q + row * K);
+  for (int64_t vi = tid; vi < nvec; vi += 256) {
+    const uint4 v = __ldcs(xr + vi);
+    qr[vi] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(v, sc);
+  }
+}
+
 }  // namespace w8a8
