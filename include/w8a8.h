@@ -191,6 +191,38 @@ W8A8_API int w8a8_last_device_error(w8a8_stream_t stream);
  */
 W8A8_API int w8a8_selftest_bounded_wait(int64_t limit_ns, w8a8_stream_t stream);
 
+/*
+ * w8a8_linear_fused for callers that cannot allocate device memory and so
+ * cannot supply a workspace: for example a plugin running inside a serving
+ * runtime or framework that reserves all device memory at start-up and
+ * forbids any later allocation, or code held to a fixed memory budget.  It
+ * computes exactly what w8a8_linear_fused computes (same arguments minus
+ * q_out / s_a_out / workspace), but keeps the int8 activations and their
+ * scales in a scratch area compiled into the library: a static device array
+ * of 16 MiB for q plus 64 KiB for the row scales.  Every GPU that loads this
+ * library holds that array until the process exits.
+ *
+ * Limits: M * K <= 16 MiB (16777216) and M <= 16384; a larger call returns
+ * W8A8_ERR_WORKSPACE and launches nothing.  It never calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ *
+ * Set-up: the first call on each device looks up the device address of the
+ * scratch array (with that device current) and caches it; make that first
+ * call before any stream capture begins.
+ *
+ * Sharing: all calls on a device use the same scratch array, which keeps
+ * whatever the previous call left there.  Each call writes the scratch it
+ * reads before reading it, so nothing needs to start at zero; but calls whose
+ * execution overlaps on the GPU (different streams, or threads that do not
+ * order their calls) race on the array -- the caller must serialize them.
+ *
+ * The paper has no counterpart to this entry point.
+ */
+W8A8_API int w8a8_linear_fused_noalloc(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                       const int8_t *Wq, const float *s_w,
+                                       const void *bias_bf16_or_null, int64_t N, void *y_bf16,
+                                       int64_t ldy, w8a8_stream_t stream);
+
 /* Library version string, e.g. "w8a8 1.0 sm_100a". */
 W8A8_API const char *w8a8_version(void);
 

@@ -71,6 +71,8 @@ _SIGNATURES = {
                            _vp, _sz, _vp], _int),
     "w8a8_linear_fused_host": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz,
                                 _vp], _int),
+    "w8a8_linear_fused_noalloc": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp],
+                                  _int),
     "w8a8_select": ([_i64, _i64, _i64, _i32, _int, ctypes.POINTER(Plan)], _int),
     "w8a8_last_device_error": ([_vp], _int),
     "w8a8_selftest_bounded_wait": ([_i64, _vp], _int),
@@ -151,6 +153,10 @@ def w8a8_linear_fused_host(x_host, M, K, Wq, s_w, bias, N, y_host, x_dev, y_dev,
                            ws_bytes, stream) -> int:
     return lib().w8a8_linear_fused_host(x_host, M, K, Wq, s_w, bias, N, y_host, x_dev, y_dev,
                                         workspace, ws_bytes, stream)
+
+
+def w8a8_linear_fused_noalloc(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, stream) -> int:
+    return lib().w8a8_linear_fused_noalloc(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, stream)
 
 
 def w8a8_select(M, N, K, num_sms=148, variant=VARIANT_AUTO) -> tuple[int, Plan]:

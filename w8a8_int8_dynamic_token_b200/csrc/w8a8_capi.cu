@@ -9,6 +9,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/w8a8.h"
 #include "w8a8_gemm.cuh"
@@ -347,6 +348,49 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
                                                           y, ldy, acc, stream);
 }
 
+// ---------------------------------------------------------------- static scratch
+// Scratch for w8a8_linear_fused_noalloc: the int8 activations (up to 16 MiB)
+// followed by their fp32 row scales (up to 16384 rows).  In host code the
+// array's name only stands in for the device object; its device address is
+// looked up once per device with cudaGetSymbolAddress.
+constexpr size_t kNoAllocMaxQBytes = static_cast<size_t>(16) << 20;
+constexpr int64_t kNoAllocMaxRows = 16384;
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocMaxQBytes + static_cast<size_t>(kNoAllocMaxRows) * sizeof(float);
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocScratch {
+  std::atomic<int> state{0};  // 1 once ptr holds this device's address
+  void *ptr = nullptr;
+  std::mutex mu;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
+// Device address of the scratch array on the current device (looked up on
+// the first call per device).
+int noalloc_scratch(void **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  NoAllocScratch &s = g_noalloc[dev];
+  if (s.state.load(std::memory_order_acquire) != 1) {
+    std::lock_guard<std::mutex> lock(s.mu);
+    if (s.state.load(std::memory_order_relaxed) != 1) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return W8A8_ERR_CUDA;
+      }
+      s.ptr = p;
+      s.state.store(1, std::memory_order_release);
+    }
+  }
+  *out = s.ptr;
+  return W8A8_OK;
+}
+
 }  // namespace w8a8
 
 using namespace w8a8;
@@ -487,6 +531,26 @@ int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const in
   st = launch_quant(x, M, K, ldx, q, s_a, stream);
   if (st != W8A8_OK) return st;
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, nullptr, plan.variant, stream);
+}
+
+int w8a8_linear_fused_noalloc(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t *Wq,
+                              const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
+                              w8a8_stream_t stream) {
+  if (!x || !Wq || !s_w || !y) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(M, K, ldx);
+  if (st != W8A8_OK) return st;
+  st = check_n(N, ldy);
+  if (st != W8A8_OK) return st;
+  if (M > kNoAllocMaxRows || M * K > static_cast<int64_t>(kNoAllocMaxQBytes))
+    return W8A8_ERR_WORKSPACE;  // beyond the static scratch limits
+  const DeviceInfo *d = nullptr;
+  st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  void *scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != W8A8_OK) return st;
+  return w8a8_linear_fused(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, nullptr, nullptr, scratch,
+                           kNoAllocScratchBytes, stream);
 }
 
 int w8a8_linear_fused_host(const void *x_host, int64_t M, int64_t K, const int8_t *Wq,
