@@ -94,6 +94,15 @@ def test_quant_edge_rows(K):
     assert q_ref[4].min() == 127                                # all-equal subnormal row
 
 
+def test_division_free_quant_step_exhaustive():
+    # every positive finite bf16 row maximum a with every bf16 x, |x| <= a
+    checked, bad = w8a8.binding.selftest_quant_exhaustive()
+    assert bad == 0
+    # pairs on the fast step: all maxima except the tiniest (whose scale is
+    # below 2^-100 and which take the IEEE-division path)
+    assert checked > 900_000_000
+
+
 @pytest.mark.parametrize("N,K", [(264, 3072), (128, 256), (8, 16), (520, 12288)])
 def test_quantize_weights_bitexact(N, K):
     w = synth.make_w(N, K, seed=N)

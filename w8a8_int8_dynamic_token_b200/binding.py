@@ -13,6 +13,7 @@ or PyTorch fallback: if libw8a8.so is missing this module raises on first use.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import re
 
@@ -76,6 +77,7 @@ _SIGNATURES = {
     "w8a8_select": ([_i64, _i64, _i64, _i32, _int, ctypes.POINTER(Plan)], _int),
     "w8a8_last_device_error": ([_vp], _int),
     "w8a8_selftest_bounded_wait": ([_i64, _vp], _int),
+    "w8a8_selftest_quant_exhaustive": ([_vp, _vp], _int),
 }
 
 
@@ -199,6 +201,7 @@ def _need(t, name, dtype, ndim, device=None):
         raise ValueError(f"{name} must have unit stride in its last dimension")
 
 
+@functools.lru_cache(maxsize=1024)
 def workspace_size(M: int, N: int, K: int) -> int:
     st, n = w8a8_workspace_size(M, N, K)
     _check(st, "w8a8_workspace_size")
@@ -321,3 +324,17 @@ def last_device_error(stream=None) -> int:
 
 def selftest_bounded_wait(limit_ns: int, stream=None) -> int:
     return w8a8_selftest_bounded_wait(int(limit_ns), _stream(stream))
+
+
+def w8a8_selftest_quant_exhaustive(counts_dev, stream) -> int:
+    return lib().w8a8_selftest_quant_exhaustive(counts_dev, stream)
+
+
+def selftest_quant_exhaustive(stream=None) -> tuple[int, int]:
+    """(pairs checked, pairs whose code differs from the IEEE-division path)."""
+    counts = torch.zeros(2, dtype=torch.int64, device="cuda")
+    _check(w8a8_selftest_quant_exhaustive(_ptr(counts), _stream(stream)),
+           "w8a8_selftest_quant_exhaustive")
+    torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+    c = counts.cpu().tolist()
+    return int(c[0]), int(c[1])

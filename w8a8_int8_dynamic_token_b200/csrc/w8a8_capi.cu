@@ -24,6 +24,8 @@ constexpr int kMaxDevices = 64;
 constexpr int kGemmStages256 = 4;  // 4 x 48 KB ring for 128x256 tiles
 constexpr int kGemmStages128 = 6;  // 6 x 32 KB ring for 128x128 tiles
 constexpr int kGemmGroupM = 8;
+constexpr int64_t kQuantMaxV = 12;  // 16-byte vectors per thread in the quant kernel
+constexpr int kGemvMaxSmem = 232448 - 1024;   // q rows of the GEMV (M * K bytes)
 
 // ---------------------------------------------------------------- device info
 
@@ -111,8 +113,8 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     if (!gemv_fits(M, K, max_smem)) return W8A8_ERR_UNSUPPORTED_SHAPE;
     const int64_t smem = M * K;
     int per_sm = static_cast<int>((max_smem) / (smem + 1024));
-    per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
-    const int64_t rows_per_cta = kGemvThreads / 32;
+    per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+    const int64_t rows_per_cta = kGemvWarps * kGemvRows;
     int64_t grid = cdiv(N, rows_per_cta);
     const int64_t cap = static_cast<int64_t>(sms) * per_sm;
     plan->num_tiles = static_cast<int32_t>(N);
@@ -165,6 +167,22 @@ int encode_i8_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, i
   return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
 }
 
+// bf16 matrix [rows, cols] with row stride ld elements, box 32 x 32, 64-byte
+// swizzle (the epilogue's staging layout).
+int encode_bf16_store_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols,
+                          int64_t ld) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return W8A8_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kEpiChunk), 32u};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- launches
 
 template <typename... KArgs, typename... Args>
@@ -185,48 +203,61 @@ int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStr
   return W8A8_OK;
 }
 
-template <typename K>
-int set_smem_attr(K kernel, int bytes) {
-  if (cudaFuncSetAttribute(reinterpret_cast<const void *>(kernel),
+// Raise a kernel's dynamic shared memory limit to `bytes`, once per device
+// (the attribute is per function and device; setting it costs microseconds,
+// so it is not repeated on every call).  Each kernel asks for its largest
+// possible footprint.
+template <auto Kernel>
+int ensure_smem_limit(int bytes) {
+  static std::atomic<uint64_t> done{0};  // one bit per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return W8A8_OK;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void *>(Kernel),
                            cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
     cudaGetLastError();
     return W8A8_ERR_CUDA;
   }
+  done.fetch_or(bit, std::memory_order_acq_rel);
   return W8A8_OK;
 }
 
 int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q, float *s,
-                 cudaStream_t stream) {
-  // G threads per row (32..256) holding V <= 8 vectors of 8 bf16 each in
-  // registers; longer rows take the two-pass kernel.
+                 int sms, cudaStream_t stream) {
+  (void)sms;
+  const uint16_t *xp = static_cast<const uint16_t *>(x);
+  if (rows > INT32_MAX / 2) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  // G threads per row (32 .. 256), each holding V <= kQuantMaxV vectors of
+  // 8 bf16 in registers; longer rows take the two-pass kernel.
   const int64_t nvec = K / 8;
   int G = 32;
   int64_t V = cdiv(nvec, G);
-  while (V > 8 && G < 256) {
+  while (V > kQuantMaxV && G < 256) {
     G *= 2;
     V = cdiv(nvec, G);
   }
-  const uint16_t *xp = static_cast<const uint16_t *>(x);
-  if (rows > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
-  if (V > 8) {
+  if (V > kQuantMaxV) {  // rows longer than 256 x 12 x 8 = 24576 elements
     return launch(quant_rows_long_kernel, dim3(static_cast<unsigned>(rows)), dim3(256), 0, stream,
                   xp, K, ldx, q, s);
   }
-  const int block = 256;
-  const int rows_per_block = block / G;
+  const int rows_per_block = 256 / G;
   const int64_t grid = cdiv(rows, rows_per_block);
-#define W8A8_QUANT_CASE(VV)                                                                   \
-  return launch(quant_rows_kernel<VV>, dim3(static_cast<unsigned>(grid)), dim3(block), 0,     \
-                stream, xp, rows, K, ldx, q, s, G)
+  const int r32 = static_cast<int>(rows), k32 = static_cast<int>(K);
+#define W8A8_QUANT_CASE(VV)                                                                \
+  return launch(quant_rows_kernel<VV>, dim3(static_cast<unsigned>(grid)), dim3(256), 0,     \
+                stream, xp, r32, k32, ldx, q, s, G)
   switch (V) {
     case 1: W8A8_QUANT_CASE(1);
     case 2: W8A8_QUANT_CASE(2);
     case 3: W8A8_QUANT_CASE(3);
     case 4: W8A8_QUANT_CASE(4);
-    case 5: W8A8_QUANT_CASE(5);
-    case 6: W8A8_QUANT_CASE(6);
-    case 7: W8A8_QUANT_CASE(7);
-    default: W8A8_QUANT_CASE(8);
+    case 5: case 6: W8A8_QUANT_CASE(6);
+    case 7: case 8: W8A8_QUANT_CASE(8);
+    default: W8A8_QUANT_CASE(12);
   }
 #undef W8A8_QUANT_CASE
 }
@@ -236,11 +267,17 @@ int launch_gemm_t(const w8a8_plan &plan, const int8_t *q, const float *s_a, int6
                   int64_t K, const int8_t *wq, const float *s_w, const void *bias, int64_t N,
                   void *y, int64_t ldy, int32_t *acc, cudaStream_t stream) {
   using L = GemmLayout<BN, STAGES>;
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, my;
   int st = encode_i8_map(&ma, q, M, K, kBM);
   if (st != W8A8_OK) return st;
   st = encode_i8_map(&mb, wq, N, K, BN);
   if (st != W8A8_OK) return st;
+  if (RAW) {
+    std::memset(&my, 0, sizeof(my));  // the raw-int32 variant stores directly
+  } else {
+    st = encode_bf16_store_map(&my, y, M, N, ldy);
+    if (st != W8A8_OK) return st;
+  }
   GemmParams p;
   p.M = static_cast<int32_t>(M);
   p.N = static_cast<int32_t>(N);
@@ -256,10 +293,11 @@ int launch_gemm_t(const w8a8_plan &plan, const int8_t *q, const float *s_a, int6
   p.y = static_cast<uint16_t *>(y);
   p.ldy = ldy;
   p.acc_out = acc;
-  auto kernel = gemm_i8_tcgen05_kernel<BN, STAGES, RAW>;
-  st = set_smem_attr(kernel, L::kSmemBytes);
+  constexpr auto kernel = gemm_i8_tcgen05_kernel<BN, STAGES, RAW>;
+  st = ensure_smem_limit<kernel>(L::kSmemBytes);
   if (st != W8A8_OK) return st;
-  return launch(kernel, dim3(plan.grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma, mb, p);
+  return launch(kernel, dim3(plan.grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma, mb, my,
+                p);
 }
 
 template <bool FUSED, bool RAW>
@@ -269,8 +307,8 @@ int launch_gemv_m(const w8a8_plan &plan, const GemvParams &p, int max_smem,
   (void)max_smem;
 #define W8A8_GEMV_CASE(MT)                                                              \
   {                                                                                     \
-    auto kernel = gemv_i8_kernel<MT, FUSED, RAW>;                                       \
-    int st = set_smem_attr(kernel, smem);                                               \
+    constexpr auto kernel = gemv_i8_kernel<MT, FUSED, RAW>;                             \
+    int st = ensure_smem_limit<kernel>(kGemvMaxSmem);                                   \
     if (st != W8A8_OK) return st;                                                       \
     return launch(kernel, dim3(plan.grid), dim3(kGemvThreads), smem, stream, p);        \
   }
@@ -300,6 +338,26 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
   __syncthreads();
   // nothing ever arrives on `bar`: the wait must give up after limit_ns
   if (threadIdx.x == 0) mbar_wait(&bar, 0u, &abort_flag, limit_ns);
+}
+
+// Every positive finite bf16 maximum a (blockIdx.x + 1) against every bf16
+// value x with |x| <= a: the fast step's result must equal the IEEE-division
+// path's, bit for bit.
+__global__ void __launch_bounds__(256) quant_exhaustive_kernel(unsigned long long *counts) {
+  const uint32_t abits = blockIdx.x + 1u;  // 0x0001 .. 0x7F7F
+  const float a = __uint_as_float(abits << 16);
+  const float s = __fdiv_rn(a, 127.0f);
+  if (!quant_fast_ok(s)) return;
+  const float y = __frcp_rn(s);
+  unsigned long long checked = 0, bad = 0;
+  for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
+    if ((xb & 0x7FFFu) > abits) continue;  // |x| > a (also skips Inf and NaN)
+    const float x = __uint_as_float(xb << 16);
+    ++checked;
+    if (quant_fast(x, s, y) != quant_exact(x, s)) ++bad;
+  }
+  atomicAdd(&counts[0], checked);
+  if (bad) atomicAdd(&counts[1], bad);
 }
 
 int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
@@ -423,7 +481,7 @@ int w8a8_quantize_weights(const void *W, int64_t N, int64_t K, int64_t ldw, int8
   const DeviceInfo *d = nullptr;
   st = query_device(&d);
   if (st != W8A8_OK) return st;
-  return launch_quant(W, N, K, ldw, Wq, s_w, reinterpret_cast<cudaStream_t>(stream));
+  return launch_quant(W, N, K, ldw, Wq, s_w, d->sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q, float *s_a,
@@ -436,7 +494,7 @@ int w8a8_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q, 
   const DeviceInfo *d = nullptr;
   st = query_device(&d);
   if (st != W8A8_OK) return st;
-  return launch_quant(x, M, K, ldx, q, s_a, reinterpret_cast<cudaStream_t>(stream));
+  return launch_quant(x, M, K, ldx, q, s_a, d->sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_select(int64_t M, int64_t N, int64_t K, int32_t num_sms, int variant,
@@ -528,7 +586,7 @@ int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const in
     if (!q) q = reinterpret_cast<int8_t *>(ws);
     if (!s_a) s_a = reinterpret_cast<float *>(ws + align256(static_cast<size_t>(M * K)));
   }
-  st = launch_quant(x, M, K, ldx, q, s_a, stream);
+  st = launch_quant(x, M, K, ldx, q, s_a, d->sms, stream);
   if (st != W8A8_OK) return st;
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, nullptr, plan.variant, stream);
 }
@@ -594,6 +652,19 @@ int w8a8_last_device_error(w8a8_stream_t stream) {
     return W8A8_ERR_CUDA;
   }
   return (word & W8A8_DEVERR_TIMEOUT) ? W8A8_ERR_DEVICE_TIMEOUT : W8A8_OK;
+}
+
+int w8a8_selftest_quant_exhaustive(unsigned long long *counts_dev, w8a8_stream_t stream_) {
+  if (!counts_dev) return W8A8_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const DeviceInfo *d = nullptr;
+  int st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  if (cudaMemsetAsync(counts_dev, 0, 2 * sizeof(unsigned long long), stream) != cudaSuccess) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  return launch(quant_exhaustive_kernel, dim3(0x7F7F), dim3(256), 0, stream, counts_dev);
 }
 
 int w8a8_selftest_bounded_wait(int64_t limit_ns, w8a8_stream_t stream) {

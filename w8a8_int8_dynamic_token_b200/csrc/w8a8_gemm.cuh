@@ -19,12 +19,17 @@
 //               K=32 per instruction) into one of two TMEM accumulators, then
 //               commits to the ring's "empty" barriers and the accumulator's
 //               "full" barrier;
-//   warps 2..5  the epilogue: tcgen05.ld of the accumulator (each warp owns
-//               the 32 TMEM lanes = rows its warp index selects), the fp32
-//               scale/bias math, bf16 packing and 16-byte stores; then they
-//               release the accumulator so the next tile's MMAs overlap them.
-// Ragged edges: TMA zero-fills rows/columns outside the tensors (zeros add
-// nothing to an integer dot product); the epilogue masks its stores.
+//   warps 2..9  the epilogue, two warps per 32-lane TMEM quarter (a warp may
+//               only read the quarter its index selects), each taking half of
+//               the tile's columns in chunks of 32: tcgen05.ld, the fp32
+//               scale/bias math, bf16 packing into a 64-byte-swizzled staging
+//               buffer in shared memory, and a TMA store of the 32 x 32 box
+//               (two staging buffers per warp, so the store of one chunk
+//               overlaps the math of the next).  After its last chunk a warp
+//               releases the accumulator, so the next tile's MMAs overlap the
+//               epilogue of this one.
+// Ragged edges: TMA zero-fills rows/columns outside the tensors on load (zeros
+// add nothing to an integer dot product) and clips them on store.
 #pragma once
 
 #include <cuda.h>
@@ -35,7 +40,10 @@
 
 namespace w8a8 {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;   // 2 + 8 warps
+constexpr int kEpiWarps = 8;
+constexpr int kEpiChunk = 32;        // columns per epilogue step
+constexpr int kEpiBufBytes = 32 * kEpiChunk * 2;  // 32 rows x 32 bf16
 constexpr int kBM = 128;   // rows of y per tile (TMEM lanes)
 constexpr int kBK = 128;   // int8 K elements per stage = one 128-byte swizzle row
 constexpr int kMmaK = 32;  // K per tcgen05.mma kind::i8
@@ -46,10 +54,14 @@ struct GemmLayout {
   static constexpr int kBBytes = BN * kBK;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTileBytes = STAGES * kStageBytes;
+  static constexpr int kEpiOffset = kTileBytes;  // 1024-aligned
+  static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiBufBytes;
+  static constexpr int kBarOffset = kEpiOffset + kEpiBytes;
   // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, then two words
   static constexpr int kBarBytes = (2 * STAGES + 5) * 8 + 8;
-  static constexpr int kSmemBytes = kTileBytes + kBarBytes + 1024;  // + alignment slack
+  static constexpr int kSmemBytes = kBarOffset + kBarBytes + 1024;  // + alignment slack
   static constexpr int kTmemCols = 2 * BN;                          // two accumulators
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct GemmParams {
@@ -85,12 +97,13 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) 
 template <int BN, int STAGES, bool RAW_OUT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                           const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
+                           const __grid_constant__ CUtensorMap tmap_b,
+                           const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
   using L = GemmLayout<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kTileBytes);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBarOffset);
   uint64_t *empty = full + STAGES;
   uint64_t *tfull = empty + STAGES;
   uint64_t *tempty = tfull + 2;
@@ -108,13 +121,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[a], kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
+    if constexpr (!RAW_OUT) tma_prefetch_desc(&tmap_y);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
@@ -212,30 +226,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 = tile rows
+    const int e = warp - 2;            // 0..7
+    const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31 = tile rows
+    const int half = e >> 2;           // which half of the tile's columns
+    constexpr int kCols = BN / 2;      // columns per warp
+    uint8_t *stage_buf = smem + L::kEpiOffset + e * 2 * kEpiBufBytes;
+    uint32_t chunk_count = 0;          // TMA stores issued by this warp
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
       int mb, nb;
       gemm_tile_coords(t, p, mb, nb);
+      const int row0 = mb * kBM + quarter * 32;
+      const int row = row0 + lane;
+      const bool row_ok = row < p.M;
+      const float sa = row_ok ? __ldg(p.s_a + row) : 0.0f;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], acc_phase, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-
-      const int row = mb * kBM + quarter * 32 + lane;
-      const bool row_ok = row < p.M;
-      const float sa = row_ok ? __ldg(p.s_a + row) : 0.0f;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
+                             static_cast<uint32_t>(acc * BN + half * kCols);
+      // a warp whose 32 rows all lie past M has nothing to store
+      const int cols_here = row0 < p.M ? kCols : 0;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + c, r);
-        tmem_ld_wait();
-        const int col0 = nb * BN + c;
+      for (int c = 0; c < cols_here; c += kEpiChunk) {
+        const int col0 = nb * BN + half * kCols + c;
+        if (col0 >= p.N) break;  // warp-uniform
         if constexpr (RAW_OUT) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + c, r);
+          tmem_ld_wait();
           if (row_ok) {
             int32_t *dst = p.acc_out + static_cast<int64_t>(row) * p.N + col0;
 #pragma unroll
@@ -247,43 +269,68 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         } else {
-          uint16_t *dst = p.y + static_cast<int64_t>(row) * p.ldy + col0;
+          // per-column scale and bias of this chunk (warp-uniform addresses);
+          // issued before the TMEM load so the two latencies overlap
+          float sw[32];
+          uint32_t bw[16];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {  // 8 columns per group; N % 8 == 0
+          for (int g = 0; g < 4; ++g) {
             const int cg = col0 + 8 * g;
-            if (cg >= p.N) break;
-            const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg));
-            const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg) + 1);
-            const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            float bb[8];
-            if (p.bias != nullptr) {
-              const uint4 braw = __ldg(reinterpret_cast<const uint4 *>(p.bias + cg));
-              const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                bb[2 * i] = __uint_as_float(bw[i] << 16);
-                bb[2 * i + 1] = __uint_as_float(bw[i] & 0xFFFF0000u);
-              }
-            }
-            uint32_t packed[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              float v0 = __int2float_rn(static_cast<int32_t>(r[8 * g + 2 * i]));
-              float v1 = __int2float_rn(static_cast<int32_t>(r[8 * g + 2 * i + 1]));
-              v0 = __fmul_rn(__fmul_rn(v0, sa), sw[2 * i]);
-              v1 = __fmul_rn(__fmul_rn(v1, sa), sw[2 * i + 1]);
+            if (cg < p.N) {
+              const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg));
+              const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg) + 1);
+              sw[8 * g + 0] = w0.x; sw[8 * g + 1] = w0.y; sw[8 * g + 2] = w0.z; sw[8 * g + 3] = w0.w;
+              sw[8 * g + 4] = w1.x; sw[8 * g + 5] = w1.y; sw[8 * g + 6] = w1.z; sw[8 * g + 7] = w1.w;
               if (p.bias != nullptr) {
-                v0 = __fadd_rn(v0, bb[2 * i]);
-                v1 = __fadd_rn(v1, bb[2 * i + 1]);
+                const uint4 braw = __ldg(reinterpret_cast<const uint4 *>(p.bias + cg));
+                bw[4 * g + 0] = braw.x; bw[4 * g + 1] = braw.y;
+                bw[4 * g + 2] = braw.z; bw[4 * g + 3] = braw.w;
+              } else {
+                bw[4 * g + 0] = bw[4 * g + 1] = bw[4 * g + 2] = bw[4 * g + 3] = 0u;
               }
-              const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-              packed[i] = *reinterpret_cast<const uint32_t *>(&h);
-            }
-            if (row_ok) {
-              reinterpret_cast<uint4 *>(dst)[g] =
-                  make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) sw[8 * g + i] = 0.0f;
+              bw[4 * g + 0] = bw[4 * g + 1] = bw[4 * g + 2] = bw[4 * g + 3] = 0u;
             }
           }
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + c, r);
+          tmem_ld_wait();
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float v0 = __int2float_rn(static_cast<int32_t>(r[2 * i]));
+            float v1 = __int2float_rn(static_cast<int32_t>(r[2 * i + 1]));
+            v0 = __fmul_rn(__fmul_rn(v0, sa), sw[2 * i]);
+            v1 = __fmul_rn(__fmul_rn(v1, sa), sw[2 * i + 1]);
+            if (p.bias != nullptr) {
+              v0 = __fadd_rn(v0, __uint_as_float(bw[i] << 16));
+              v1 = __fadd_rn(v1, __uint_as_float(bw[i] & 0xFFFF0000u));
+            }
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+            packed[i] = *reinterpret_cast<const uint32_t *>(&h);
+          }
+          // staging buffer of this chunk: free once the store issued two
+          // chunks ago has finished reading it
+          uint8_t *buf = stage_buf + (chunk_count & 1u) * kEpiBufBytes;
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          // row `lane` = 64 bytes = four 16-byte pieces; 64-byte swizzle:
+          // piece j of row r sits at position j ^ ((r >> 1) & 3)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int pos = j ^ ((lane >> 1) & 3);
+            *reinterpret_cast<uint4 *>(buf + lane * 64 + pos * 16) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmap_y, buf, col0, row0);
+            bulk_commit_group();
+          }
+          ++chunk_count;
         }
       }
       tc_fence_before();
@@ -293,6 +340,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc = 0;
         acc_phase ^= 1u;
       }
+    }
+    if constexpr (!RAW_OUT) {
+      if (lane == 0) bulk_wait_all();  // staging buffers stay valid until stored
+      __syncwarp();
     }
   }
 

@@ -9,9 +9,11 @@
 //   1. (fused variant) every CTA quantizes the M activation rows into shared
 //      memory with the per-token rule of the quantization kernel;
 //      (unfused variant) every CTA copies the given q rows into shared memory;
-//   2. each warp walks whole weight rows n, lanes reading 16-byte vectors with
-//      evict-first loads, accumulating M int32 dot products with dp4a
-//      (exact: every partial sum is bounded by 127*127*K < 2^31);
+//   2. each warp walks pairs of weight rows, every lane holding 8 16-byte
+//      vectors of each row in flight (evict-first loads; the first pair's
+//      loads are issued before step 1 so the prologue hides under them),
+//      accumulating M int32 dot products with dp4a (exact: every partial sum
+//      is bounded by 127*127*K < 2^31);
 //   3. a warp reduction, then lane m writes
 //      y[m,n] = bf16_rne(((float)acc * s_a[m]) * s_w[n] + (float)bias[n]).
 #pragma once
@@ -42,7 +44,7 @@ struct GemvParams {
   float *s_a_out;     // fused variant: optional copy of s_a
 };
 
-// Block-wide max of non-negative 16-bit patterns.
+// Block-wide max of bit patterns of non-negative floats.
 __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
@@ -56,38 +58,64 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *red) {
   return v;
 }
 
+constexpr int kGemvWarps = kGemvThreads / 32;
+constexpr int kGemvRows = 2;  // weight rows per warp step
+constexpr int kGemvVec = 8;   // 16-byte weight vectors per lane per row per step
+
+// Loads kGemvVec 16-byte vectors per row for the rows n0, n0+1, starting at
+// vector index kb + lane (stride 32); rows past N and vectors past K read 0.
+__device__ __forceinline__ void gemv_load(const int8_t *__restrict__ wq, int N, int nvec16,
+                                          int n0, int kb, int lane,
+                                          uint4 (&wv)[kGemvRows][kGemvVec]) {
+#pragma unroll
+  for (int r = 0; r < kGemvRows; ++r) {
+    const int n = n0 + r;
+    const uint4 *wr = reinterpret_cast<const uint4 *>(wq + static_cast<int64_t>(n) * nvec16 * 16);
+#pragma unroll
+    for (int u = 0; u < kGemvVec; ++u) {
+      const int vi = kb + lane + 32 * u;
+      wv[r][u] = (n < N && vi < nvec16) ? __ldcs(wr + vi) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
 template <int MT, bool FUSED, bool RAW_OUT>
 __global__ void __launch_bounds__(kGemvThreads) gemv_i8_kernel(const GemvParams p) {
   extern __shared__ __align__(16) uint8_t gemv_smem[];
   int8_t *qs = reinterpret_cast<int8_t *>(gemv_smem);  // [M][K]
   __shared__ float sas[kGemvMaxM];
-  __shared__ uint32_t red[kGemvThreads / 32];
+  __shared__ uint32_t red[kGemvWarps];
 
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int K = p.K;
   const int nvec8 = K >> 3;    // 8-element bf16 vectors per row
   const int nvec16 = K >> 4;   // 16-byte int8 vectors per row
+  const int npairs = (p.N + kGemvRows - 1) / kGemvRows;
+  const int warps_total = gridDim.x * kGemvWarps;
+  int pi = blockIdx.x * kGemvWarps + warp;
+
+  // The weight stream is what this kernel waits on: start it before the
+  // activation prologue.
+  uint4 wv[kGemvRows][kGemvVec];
+  if (pi < npairs) gemv_load(p.wq, p.N, nvec16, pi * kGemvRows, 0, lane, wv);
 
   // ---- 1. activation rows -> shared memory (int8) + scales
   if constexpr (FUSED) {
     for (int m = 0; m < p.M; ++m) {
       const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(m) * p.ldx);
-      uint32_t mm = 0u;
-      for (int v = tid; v < nvec8; v += kGemvThreads) {
-        const uint4 a = __ldg(xr + v);
-        mm = bf16x2_absmax(mm, a.x);
-        mm = bf16x2_absmax(mm, a.y);
-        mm = bf16x2_absmax(mm, a.z);
-        mm = bf16x2_absmax(mm, a.w);
-      }
-      const uint32_t mb = block_max_u32(bf16x2_max_halves(mm), red);
-      const float amax = __uint_as_float(mb << 16);
+      float mm = 0.0f;
+      for (int v = tid; v < nvec8; v += kGemvThreads) mm = absmax_vec8(__ldg(xr + v), mm);
+      const uint32_t mb = block_max_u32(__float_as_uint(mm), red);
+      const float amax = __uint_as_float(mb);
       const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+      const bool fast = quant_fast_ok(sc);
+      const float rc = fast ? __frcp_rn(sc) : 0.0f;
       if (tid == 0) sas[m] = sc;
       uint2 *qrow = reinterpret_cast<uint2 *>(qs + m * K);
       for (int v = tid; v < nvec8; v += kGemvThreads) {
         const uint4 a = __ldg(xr + v);
-        qrow[v] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(a, sc);
+        qrow[v] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(a, sc, rc, fast);
       }
     }
   } else {
@@ -108,58 +136,62 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_i8_kernel(const GemvParams 
     }
   }
 
-  // ---- 2. stream weight rows
-  const int warp = tid >> 5, lane = tid & 31;
-  const int warps_total = gridDim.x * (kGemvThreads / 32);
-  constexpr int U = 4;  // 16-byte weight vectors in flight per lane
-  for (int n = blockIdx.x * (kGemvThreads / 32) + warp; n < p.N; n += warps_total) {
-    const uint4 *wr = reinterpret_cast<const uint4 *>(p.wq + static_cast<int64_t>(n) * K);
-    int acc[MT];
+  // ---- 2. stream weight rows, two rows per warp step
+  bool loaded = true;  // wv already holds (pi, kb = 0)
+  for (; pi < npairs; pi += warps_total) {
+    const int n0 = pi * kGemvRows;
+    int acc[kGemvRows][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0;
-    for (int base = lane; base < nvec16; base += 32 * U) {
-      uint4 wv[U];
+    for (int r = 0; r < kGemvRows; ++r)
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int vi = base + 32 * u;
-        wv[u] = vi < nvec16 ? __ldcs(wr + vi) : make_uint4(0u, 0u, 0u, 0u);
-      }
+      for (int m = 0; m < MT; ++m) acc[r][m] = 0;
+    for (int kb = 0; kb < nvec16; kb += 32 * kGemvVec) {
+      if (!loaded) gemv_load(p.wq, p.N, nvec16, n0, kb, lane, wv);
+      loaded = false;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int vi = base + 32 * u;
+      for (int u = 0; u < kGemvVec; ++u) {
+        const int vi = kb + lane + 32 * u;
         if (vi < nvec16) {
 #pragma unroll
           for (int m = 0; m < MT; ++m) {
             if (m < p.M) {
               const int4 qv = reinterpret_cast<const int4 *>(qs + m * K)[vi];
-              acc[m] = __dp4a(static_cast<int>(wv[u].x), qv.x, acc[m]);
-              acc[m] = __dp4a(static_cast<int>(wv[u].y), qv.y, acc[m]);
-              acc[m] = __dp4a(static_cast<int>(wv[u].z), qv.z, acc[m]);
-              acc[m] = __dp4a(static_cast<int>(wv[u].w), qv.w, acc[m]);
+#pragma unroll
+              for (int r = 0; r < kGemvRows; ++r) {
+                acc[r][m] = __dp4a(static_cast<int>(wv[r][u].x), qv.x, acc[r][m]);
+                acc[r][m] = __dp4a(static_cast<int>(wv[r][u].y), qv.y, acc[r][m]);
+                acc[r][m] = __dp4a(static_cast<int>(wv[r][u].z), qv.z, acc[r][m]);
+                acc[r][m] = __dp4a(static_cast<int>(wv[r][u].w), qv.w, acc[r][m]);
+              }
             }
           }
         }
       }
     }
-    // ---- 3. reduce across the warp, lane m finishes row m
+    // ---- 3. reduce across the warp; lane m finishes row m of each weight row
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
+    for (int r = 0; r < kGemvRows; ++r) {
+      const int n = n0 + r;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[m] += __shfl_xor_sync(0xFFFFFFFFu, acc[m], o);
-    }
-    int mine = 0;
+      for (int m = 0; m < MT; ++m) {
 #pragma unroll
-    for (int m = 0; m < MT; ++m)
-      if (lane == m) mine = acc[m];
-    if (lane < p.M) {
-      if constexpr (RAW_OUT) {
-        p.acc_out[static_cast<int64_t>(lane) * p.N + n] = mine;
-      } else {
-        float v = __int2float_rn(mine);
-        v = __fmul_rn(__fmul_rn(v, sas[lane]), __ldg(p.s_w + n));
-        if (p.bias != nullptr) v = __fadd_rn(v, __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16));
-        const __nv_bfloat16 h = __float2bfloat16_rn(v);
-        p.y[static_cast<int64_t>(lane) * p.ldy + n] = *reinterpret_cast<const uint16_t *>(&h);
+        for (int o = 16; o > 0; o >>= 1) acc[r][m] += __shfl_xor_sync(0xFFFFFFFFu, acc[r][m], o);
+      }
+      int mine = 0;
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (lane == m) mine = acc[r][m];
+      if (lane < p.M && n < p.N) {
+        if constexpr (RAW_OUT) {
+          p.acc_out[static_cast<int64_t>(lane) * p.N + n] = mine;
+        } else {
+          float v = __int2float_rn(mine);
+          v = __fmul_rn(__fmul_rn(v, sas[lane]), __ldg(p.s_w + n));
+          if (p.bias != nullptr)
+            v = __fadd_rn(v, __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16));
+          const __nv_bfloat16 h = __float2bfloat16_rn(v);
+          p.y[static_cast<int64_t>(lane) * p.ldy + n] = *reinterpret_cast<const uint16_t *>(&h);
+        }
       }
     }
   }

@@ -10,127 +10,120 @@
 //                                             rint: nearest, ties to even
 //   max |x| == 0  ->  s = 0, q = 0
 //
-// Layout of the work: a group of G threads owns one row.  Each thread loads V
-// 16-byte vectors (8 bf16 each) of the row into registers with streaming
-// loads, so the row is read from HBM exactly once; the group reduces max |x|
-// as an integer max of bit patterns (packed 16-bit max, warp shuffles and,
-// for G > 32, shared memory); then every
-// thread quantizes its registers and writes 8 int8 per vector.
+// Layout of the work (quant_rows_kernel): a group of G threads owns one row,
+// keeps its vectors (8 bf16 each) in registers, reduces max |x| (fmaxf on the
+// widened values, then an integer max of the non-negative bit patterns across
+// lanes and, for G > 32, across warps through shared memory), then quantizes
+// its registers and writes 8 int8 per vector.  Each row is read from HBM
+// exactly once.
 //
-// Rounding: rint(t) for |t| <= 127.0001 is formed exactly by adding and
-// subtracting 1.5 * 2^23 in round-to-nearest-even fp32 arithmetic; the low
-// byte of (t + 1.5 * 2^23)'s bit pattern is then the two's-complement int8.
+// Rounding: rint(t) for |t| <= 127.0001 is formed exactly by adding
+// 1.5 * 2^23 in round-to-nearest-even fp32 arithmetic; the low byte of the
+// sum's bit pattern is then the two's-complement int8.  The quotient x / s is
+// not divided out element by element: the row's correctly rounded reciprocal
+// and one correction step give the same correctly rounded quotient as an IEEE
+// division, without a branch (see quant_fast).
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cstdint>
 
+
 namespace w8a8 {
 
 constexpr float kRintMagic = 12582912.0f;  // 1.5 * 2^23
 
-// Quantize two bf16 (packed in one 32-bit word) with scale s; returns the two
-// int8 codes in the low bytes of two words (as bit patterns of t + magic).
-__device__ __forceinline__ void quant_pair(uint32_t packed, float s, uint32_t &c0, uint32_t &c1) {
-  const float v0 = __uint_as_float(packed << 16);
-  const float v1 = __uint_as_float(packed & 0xFFFF0000u);
-  float t0 = __fdiv_rn(v0, s);
-  float t1 = __fdiv_rn(v1, s);
-  t0 = fminf(fmaxf(t0, -127.0f), 127.0f);
-  t1 = fminf(fmaxf(t1, -127.0f), 127.0f);
-  c0 = __float_as_uint(__fadd_rn(t0, kRintMagic));
-  c1 = __float_as_uint(__fadd_rn(t1, kRintMagic));
+// Exact path: q = clamp(rint(x / s), -127, 127) with an IEEE division.
+// Returns the bit pattern of rint(t) + 1.5 * 2^23, whose low byte is the code.
+__device__ __forceinline__ uint32_t quant_exact(float v, float s) {
+  float t = __fdiv_rn(v, s);
+  t = fminf(fmaxf(t, -127.0f), 127.0f);
+  return __float_as_uint(__fadd_rn(t, kRintMagic));
 }
 
-// 8 bf16 (one 16-byte vector) -> 8 int8 (8 bytes).
-__device__ __forceinline__ uint2 quant_vec8(uint4 v, float s) {
-  uint32_t c[8];
-  quant_pair(v.x, s, c[0], c[1]);
-  quant_pair(v.y, s, c[2], c[3]);
-  quant_pair(v.z, s, c[4], c[5]);
-  quant_pair(v.w, s, c[6], c[7]);
+// Fast path without a division: Markstein's correction step (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Develop. 34(1), 1990).  With y = RN(1/s), the
+// correctly rounded reciprocal, q0 = RN(x * y) is within one ulp of x/s, the
+// remainder e = x - q0 * s is exact in one fused multiply-add, and
+// q1 = RN(q0 + e * y) is the correctly rounded quotient RN(x/s) -- the same
+// value an IEEE division returns -- provided nothing overflows or underflows,
+// which quant_fast_ok guarantees for the row's scale.  Then rint(q1) is formed
+// by adding 1.5 * 2^23 (exact, ties to even), and |rint(q1)| <= 127 (the clamp
+// is inactive).  The step is checked exhaustively against the IEEE division
+// on the GPU (w8a8_selftest_quant_exhaustive: every positive bf16 row
+// maximum with every bf16 value of the row).
+__device__ __forceinline__ uint32_t quant_fast(float x, float s, float y) {
+  const float q0 = __fmul_rn(x, y);
+  const float e = __fmaf_rn(-q0, s, x);
+  const float q1 = __fmaf_rn(e, y, q0);
+  return __float_as_uint(__fadd_rn(q1, kRintMagic));
+}
+
+__device__ __forceinline__ uint2 pack_codes(const uint32_t (&c)[8]) {
   uint2 out;
   out.x = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
   out.y = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410);
   return out;
 }
 
-// max |x| on packed bf16 pairs, exactly: with the sign bit cleared, the
-// order of IEEE bit patterns is the order of the values, so a per-half
-// unsigned 16-bit max of (bits & 0x7FFF) is the max of |x| (subnormals too).
-__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t acc, uint32_t v) {
-  return __vmaxu2(acc, v & 0x7FFF7FFFu);
-}
-
-__device__ __forceinline__ uint32_t bf16x2_max_halves(uint32_t m) {
-  const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
-  return hi > lo ? hi : lo;
-}
-
-// x: [rows, K] bf16 (row stride ldx elements); q: [rows, K] int8 dense;
-// s: [rows] fp32.  Block = rows_per_block groups of G threads.
-template <int V>
-__global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t *__restrict__ x,
-                                                         int64_t rows, int64_t K, int64_t ldx,
-                                                         int8_t *__restrict__ q,
-                                                         float *__restrict__ s, int G) {
-  __shared__ uint32_t red[32];
-  const int tid = threadIdx.x;
-  const int group = tid / G;  // row within the block
-  const int t = tid % G;      // thread within the row group
-  const int rows_per_block = blockDim.x / G;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * rows_per_block + group;
-  const bool row_ok = row < rows;
-  const int64_t nvec = K >> 3;
-
-  const uint4 *xr = reinterpret_cast<const uint4 *>(x + (row_ok ? row : 0) * ldx);
-  uint4 v[V];
-  uint32_t m = 0u;
+// One 16-byte vector of 8 bf16 -> 8 fp32 (exact widening).
+__device__ __forceinline__ void unpack8(uint4 v, float (&x)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int j = 0; j < V; ++j) {
-    const int64_t vi = t + static_cast<int64_t>(j) * G;
-    if (row_ok && vi < nvec) {
-      v[j] = __ldcs(xr + vi);
-    } else {
-      v[j] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    m = bf16x2_absmax(m, v[j].x);
-    m = bf16x2_absmax(m, v[j].y);
-    m = bf16x2_absmax(m, v[j].z);
-    m = bf16x2_absmax(m, v[j].w);
-  }
-  // the reduction runs on the bit patterns of |x| (unsigned order = value order)
-  uint32_t mb = bf16x2_max_halves(m);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
-  if (G > 32) {
-    const int warp = tid >> 5, lane = tid & 31;
-    if (lane == 0) red[warp] = mb;
-    __syncthreads();
-    const int wpg = G >> 5;  // warps per group
-    const int first = group * wpg;
-    mb = 0u;
-    for (int w = 0; w < wpg; ++w) mb = max(mb, red[first + w]);
-  }
-  if (!row_ok) return;
-  const float amax = __uint_as_float(mb << 16);
-
-  const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
-  if (t == 0) s[row] = sc;
-  uint2 *qr = reinterpret_cast<uint2 *>(q + row * K);
-#pragma unroll
-  for (int j = 0; j < V; ++j) {
-    const int64_t vi = t + static_cast<int64_t>(j) * G;
-    if (vi < nvec) {
-      uint2 o = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(v[j], sc);
-      qr[vi] = o;
-    }
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
 }
 
-// Long rows (more than 256 threads x 8 vectors): one block of 256 threads per
-// row, two passes over the row -- max |x| first, then quantize -- the second
-// pass reading the row back from L2.
+// max(m, |x_i|): fmaxf returns one of its operands unchanged, so the maximum
+// is exact (subnormals included: nothing is compiled with flush-to-zero).
+__device__ __forceinline__ float absmax8(const float (&x)[8], float m) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+  return m;
+}
+
+// 8 bf16 (one 16-byte vector) -> 8 int8 codes (8 bytes).  s > 0; y = RN(1/s);
+// fast = the row's scale is in the range where quant_fast is exact (a
+// row-uniform choice, so there is no divergence inside a row).
+__device__ __forceinline__ uint2 quant_vec8(uint4 v, float s, float y, bool fast) {
+  float x[8];
+  unpack8(v, x);
+  uint32_t c[8];
+  if (fast) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = quant_fast(x[i], s, y);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = quant_exact(x[i], s);
+  }
+  return pack_codes(c);
+}
+
+// Per-row constants of the fast path.
+__device__ __forceinline__ bool quant_fast_ok(float s) {
+  return s >= 7.8886090522101181e-31f /* 2^-100 */ && s <= 2.6584559915698317e+36f /* 2^121 */;
+}
+
+// Largest |x| of a 16-byte vector of 8 bf16, accumulated into m.
+__device__ __forceinline__ float absmax_vec8(uint4 v, float m) {
+  float x[8];
+  unpack8(v, x);
+  return absmax8(x, m);
+}
+
+// Non-negative floats order like their bit patterns: reductions across lanes
+// run on the bits.
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// Very long rows (K > 24576): one block of 256 threads per row, two passes
+// over the row -- max |x| first, then quantize -- the second pass reading the
+// row back from L2.
 __global__ void __launch_bounds__(256) quant_rows_long_kernel(const uint16_t *__restrict__ x,
                                                               int64_t K, int64_t ldx,
                                                               int8_t *__restrict__ q,
@@ -140,29 +133,79 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const uint16_t *__
   const int tid = threadIdx.x;
   const int64_t nvec = K >> 3;
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * ldx);
-  uint32_t m = 0u;
-  for (int64_t vi = tid; vi < nvec; vi += 256) {
-    const uint4 v = __ldg(xr + vi);
-    m = bf16x2_absmax(m, v.x);
-    m = bf16x2_absmax(m, v.y);
-    m = bf16x2_absmax(m, v.z);
-    m = bf16x2_absmax(m, v.w);
-  }
-  uint32_t mb = bf16x2_max_halves(m);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+  float m = 0.0f;
+  for (int64_t vi = tid; vi < nvec; vi += 256) m = absmax_vec8(__ldg(xr + vi), m);
+  uint32_t mb = warp_max_u32(__float_as_uint(m), 32);
   if ((tid & 31) == 0) red[tid >> 5] = mb;
   __syncthreads();
   mb = 0u;
 #pragma unroll
   for (int w = 0; w < 8; ++w) mb = max(mb, red[w]);
-  const float amax = __uint_as_float(mb << 16);
+  const float amax = __uint_as_float(mb);
   const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+  const bool fast = quant_fast_ok(sc);
+  const float rc = fast ? __frcp_rn(sc) : 0.0f;
   if (tid == 0) s[row] = sc;
   uint2 *qr = reinterpret_cast<uint2 *>(q + row * K);
   for (int64_t vi = tid; vi < nvec; vi += 256) {
     const uint4 v = __ldcs(xr + vi);
-    qr[vi] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(v, sc);
+    qr[vi] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(v, sc, rc, fast);
+  }
+}
+
+// The hot-path kernel: a group of G threads owns one row (G = 32, one warp,
+// whenever the row fits in 12 vectors per lane; K = 3072 gives 12).  Each
+// thread issues all of its V 16-byte loads at once (evict-first: the
+// activations are read exactly once), reduces max |x| in registers and across
+// the group (shuffles; shared memory when G > 32), then quantizes its
+// registers with the division-free step and writes 8 int8 per vector.  The
+// row's scale needs one IEEE division and one reciprocal per warp.
+template <int V>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t *__restrict__ x,
+                                                         int rows, int K, int64_t ldx,
+                                                         int8_t *__restrict__ q,
+                                                         float *__restrict__ s, int G) {
+  __shared__ uint32_t red[8];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int group = tid / G;       // row within the block
+  const int t = tid % G;           // thread within the row group
+  const int rows_per_block = blockDim.x / G;
+  const int row = blockIdx.x * rows_per_block + group;
+  const bool row_ok = row < rows;
+  const int nvec = K >> 3;
+
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x + (row_ok ? row : 0) * ldx);
+  uint4 v[V];
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    const int vi = t + j * G;
+    v[j] = (row_ok && vi < nvec) ? __ldcs(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    if (j & 1) m1 = absmax_vec8(v[j], m1); else m0 = absmax_vec8(v[j], m0);
+  }
+  uint32_t mb = warp_max_u32(__float_as_uint(fmaxf(m0, m1)), 32);
+  if (G > 32) {  // G is uniform in the block
+    if (lane == 0) red[warp] = mb;
+    __syncthreads();
+    const int wpg = G >> 5;
+    mb = 0u;
+    for (int w = 0; w < wpg; ++w) mb = max(mb, red[group * wpg + w]);
+  }
+  if (!row_ok) return;
+  const float amax = __uint_as_float(mb);
+  const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+  const bool fast = quant_fast_ok(sc);
+  const float rc = fast ? __frcp_rn(sc) : 0.0f;
+  if (t == 0) s[row] = sc;
+  uint2 *qr = reinterpret_cast<uint2 *>(q + static_cast<int64_t>(row) * K);
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    const int vi = t + j * G;
+    if (vi < nvec) qr[vi] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(v[j], sc, rc, fast);
   }
 }
 
