@@ -108,9 +108,11 @@ def test_selector_small_m_goes_to_gemv():
 
 def test_selector_gemm_plans():
     p = w8a8.select(4352, 9216, 3072)
-    assert p["variant_name"] == "gemm_bn256" and p["num_tiles"] == 34 * 36 and p["grid"] == 148
+    assert p["variant_name"] == "gemm_pair" and p["num_tiles"] == 17 * 36 and p["grid"] == 148
+    p = w8a8.select(4352, 9216, 3072, variant=B.VARIANT_GEMM_BN256)
+    assert p["num_tiles"] == 34 * 36 and p["grid"] == 148
     p = w8a8.select(4352, 3072, 12288)
-    assert p["num_tiles"] == 34 * 12 and p["grid"] == 148
+    assert p["num_tiles"] == 17 * 12 and p["grid"] == 148
     # tiny output: few tiles, grid = tiles
     p = w8a8.select(64, 128, 256)
     assert p["grid"] == p["num_tiles"] == 1
@@ -133,7 +135,9 @@ def test_workspace_size_covers_q_and_scales():
 def test_selector_is_total_and_consistent(M, KN):
     K, N = KN
     p = w8a8.select(M, N, K)
-    assert p["variant_name"] in ("gemm_bn128", "gemm_bn256")
-    tn = p["tile_n"]
-    assert p["num_tiles"] == -(-M // 128) * -(-N // tn)
+    assert p["variant_name"] in ("gemm_bn128", "gemm_bn256", "gemm_pair")
+    tm, tn = p["tile_m"], p["tile_n"]
+    assert p["num_tiles"] == -(-M // tm) * -(-N // tn)
     assert 1 <= p["grid"] <= 148
+    if p["variant_name"] == "gemm_pair":
+        assert tm == tn == 256 and p["grid"] % 2 == 0

@@ -115,7 +115,7 @@ def test_quantize_weights_bitexact(N, K):
 
 GEMM_SHAPES = [(64, 128, 256), (300, 520, 400), (129, 264, 272), (1, 8, 16), (257, 1032, 3072),
                (128, 256, 128), (640, 768, 1024), (200, 136, 12288)]
-VARIANTS = [B.VARIANT_GEMM_BN128, B.VARIANT_GEMM_BN256]
+VARIANTS = [B.VARIANT_GEMM_BN128, B.VARIANT_GEMM_BN256, B.VARIANT_GEMM_PAIR]
 
 
 @pytest.mark.parametrize("variant", VARIANTS)
@@ -216,7 +216,7 @@ def test_gemm_variant_at_tiny_m_matches_gemv():
     ref = oracle.linear(x, wq_ref, sw_ref, b)
     args = (torch.from_numpy(ref["q"]).cuda(), torch.from_numpy(ref["s_a"]).cuda(),
             torch.from_numpy(wq_ref).cuda(), torch.from_numpy(sw_ref).cuda(), to_dev(b))
-    for v in (B.VARIANT_GEMV, B.VARIANT_GEMM_BN128, B.VARIANT_GEMM_BN256):
+    for v in (B.VARIANT_GEMV, B.VARIANT_GEMM_BN128, B.VARIANT_GEMM_BN256, B.VARIANT_GEMM_PAIR):
         y = w8a8.linear(*args, variant=v)
         torch.cuda.synchronize()
         assert check_y(bits_of(y), ref["y"], ref["y32"], f"variant {v}") == 0

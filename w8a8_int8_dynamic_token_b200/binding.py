@@ -36,7 +36,8 @@ VARIANT_AUTO = 0
 VARIANT_GEMV = 1
 VARIANT_GEMM_BN128 = 2
 VARIANT_GEMM_BN256 = 3
-VARIANT_NAMES = {0: "auto", 1: "gemv", 2: "gemm_bn128", 3: "gemm_bn256"}
+VARIANT_GEMM_PAIR = 4
+VARIANT_NAMES = {0: "auto", 1: "gemv", 2: "gemm_bn128", 3: "gemm_bn256", 4: "gemm_pair"}
 
 
 class W8A8Error(RuntimeError):

@@ -23,6 +23,7 @@ constexpr int64_t kMaxK = 133144;  // 127 * 127 * K <= 2^31 - 1
 constexpr int kMaxDevices = 64;
 constexpr int kGemmStages256 = 4;  // 4 x 48 KB ring for 128x256 tiles
 constexpr int kGemmStages128 = 6;  // 6 x 32 KB ring for 128x128 tiles
+constexpr int kGemmStagesPair = 6; // 6 x 32 KB ring per CTA for 256x256 pair tiles
 constexpr int kGemmGroupM = 8;
 constexpr int64_t kQuantMaxV = 12;  // 16-byte vectors per thread in the quant kernel
 constexpr int kGemvMaxSmem = 232448 - 1024;   // q rows of the GEMV (M * K bytes)
@@ -105,6 +106,17 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
       const double e128 = static_cast<double>(t128) / (cdiv(t128, sms) * sms) *
                           (static_cast<double>(N) / (cdiv(N, 128) * 128));
       v = (e128 > 1.15 * e256) ? W8A8_VARIANT_GEMM_BN128 : W8A8_VARIANT_GEMM_BN256;
+      // CTA pairs (256 x 256 tiles) halve each CTA's operand traffic; use
+      // them when the problem has enough rows that pair tiles fill the GPU
+      // about as well as single-CTA tiles do.
+      const int64_t pairs = sms / 2;
+      const int64_t tp = cdiv(M, 256) * cdiv(N, 256);
+      const double ep = static_cast<double>(tp) / (cdiv(tp, pairs) * pairs) *
+                        (static_cast<double>(M) / (cdiv(M, 256) * 256)) *
+                        (static_cast<double>(N) / (cdiv(N, 256) * 256));
+      const double e1 = (v == W8A8_VARIANT_GEMM_BN128 ? e128 : e256) *
+                        (static_cast<double>(M) / (cdiv(M, kBM) * kBM));
+      if (M >= 512 && sms >= 2 && ep >= 0.95 * e1) v = W8A8_VARIANT_GEMM_PAIR;
     }
   }
   std::memset(plan, 0, sizeof(*plan));
@@ -119,6 +131,18 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     const int64_t cap = static_cast<int64_t>(sms) * per_sm;
     plan->num_tiles = static_cast<int32_t>(N);
     plan->grid = static_cast<int32_t>(grid < cap ? grid : cap);
+    return W8A8_OK;
+  }
+  if (v == W8A8_VARIANT_GEMM_PAIR) {
+    if (sms < 2) return W8A8_ERR_UNSUPPORTED_SHAPE;
+    const int64_t tiles = cdiv(M, 256) * cdiv(N, 256);
+    if (tiles > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
+    const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
+    plan->tile_m = 256;
+    plan->tile_n = 256;
+    plan->num_tiles = static_cast<int32_t>(tiles);
+    plan->grid = static_cast<int32_t>(2 * pairs);
+    plan->waves_x100 = static_cast<int32_t>(100 * tiles / pairs);
     return W8A8_OK;
   }
   if (v != W8A8_VARIANT_GEMM_BN128 && v != W8A8_VARIANT_GEMM_BN256) return W8A8_ERR_INVALID_ARG;
@@ -300,6 +324,44 @@ int launch_gemm_t(const w8a8_plan &plan, const int8_t *q, const float *s_a, int6
                 p);
 }
 
+template <bool RAW>
+int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, int64_t M,
+                     int64_t K, const int8_t *wq, const float *s_w, const void *bias, int64_t N,
+                     void *y, int64_t ldy, int32_t *acc, cudaStream_t stream) {
+  using L = PairLayout<kGemmStagesPair>;
+  CUtensorMap ma, mb, my;
+  int st = encode_i8_map(&ma, q, M, K, kBM);
+  if (st != W8A8_OK) return st;
+  st = encode_i8_map(&mb, wq, N, K, kPairBN / 2);
+  if (st != W8A8_OK) return st;
+  if (RAW) {
+    std::memset(&my, 0, sizeof(my));
+  } else {
+    st = encode_bf16_store_map(&my, y, M, N, ldy);
+    if (st != W8A8_OK) return st;
+  }
+  GemmParams p;
+  p.M = static_cast<int32_t>(M);
+  p.N = static_cast<int32_t>(N);
+  p.K = static_cast<int32_t>(K);
+  p.num_m_blk = static_cast<int32_t>(cdiv(M, 256));
+  p.num_n_blk = static_cast<int32_t>(cdiv(N, kPairBN));
+  p.num_tiles = plan.num_tiles;
+  p.k_blocks = static_cast<int32_t>(cdiv(K, kBK));
+  p.group_m = kGemmGroupM / 2;
+  p.s_a = s_a;
+  p.s_w = s_w;
+  p.bias = static_cast<const uint16_t *>(bias);
+  p.y = static_cast<uint16_t *>(y);
+  p.ldy = ldy;
+  p.acc_out = acc;
+  constexpr auto kernel = gemm_i8_tcgen05_pair_kernel<kGemmStagesPair, RAW>;
+  st = ensure_smem_limit<kernel>(L::kSmemBytes);
+  if (st != W8A8_OK) return st;
+  return launch(kernel, dim3(plan.grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma, mb, my,
+                p);
+}
+
 template <bool FUSED, bool RAW>
 int launch_gemv_m(const w8a8_plan &plan, const GemvParams &p, int max_smem,
                   cudaStream_t stream) {
@@ -393,6 +455,11 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
     p.acc_out = acc;
     return acc ? launch_gemv_m<false, true>(plan, p, d->max_smem_optin, stream)
                : launch_gemv_m<false, false>(plan, p, d->max_smem_optin, stream);
+  }
+  if (plan.variant == W8A8_VARIANT_GEMM_PAIR) {
+    return acc ? launch_gemm_pair<true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc, stream)
+               : launch_gemm_pair<false>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc,
+                                         stream);
   }
   if (plan.variant == W8A8_VARIANT_GEMM_BN128) {
     return acc ? launch_gemm_t<128, kGemmStages128, true>(plan, q, s_a, M, K, Wq, s_w, bias, N,
@@ -533,7 +600,7 @@ int w8a8_linear(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
 int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
                    const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
                    int32_t *acc_debug, int variant, w8a8_stream_t stream) {
-  if (variant < W8A8_VARIANT_AUTO || variant > W8A8_VARIANT_GEMM_BN256)
+  if (variant < W8A8_VARIANT_AUTO || variant > W8A8_VARIANT_GEMM_PAIR)
     return W8A8_ERR_INVALID_ARG;
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant,
                      reinterpret_cast<cudaStream_t>(stream));

@@ -94,6 +94,104 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) 
   return mbar_wait(bar, parity, &never, kWaitLimitNs);
 }
 
+// One epilogue warp's share of an accumulator: its 32 TMEM lanes (tile rows
+// row0 .. row0+31) and COLS columns starting at output column col_base, in
+// chunks of 32 columns.  t_row addresses (first lane, first column).
+template <int COLS, bool RAW_OUT>
+__device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const CUtensorMap *tmap_y,
+                                                    uint32_t t_row, int row0, int col_base,
+                                                    uint8_t *stage_buf, uint32_t &chunk_count,
+                                                    int lane) {
+  const int row = row0 + lane;
+  const bool row_ok = row < p.M;
+  const float sa = row_ok ? __ldg(p.s_a + row) : 0.0f;
+  // a warp whose 32 rows all lie past M has nothing to store
+  const int cols_here = row0 < p.M ? COLS : 0;
+#pragma unroll 1
+  for (int c = 0; c < cols_here; c += kEpiChunk) {
+    const int col0 = col_base + c;
+    if (col0 >= p.N) break;  // warp-uniform
+    if constexpr (RAW_OUT) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(t_row + c, r);
+      tmem_ld_wait();
+      if (row_ok) {
+        int32_t *dst = p.acc_out + static_cast<int64_t>(row) * p.N + col0;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          if (col0 + 4 * g < p.N) {
+            reinterpret_cast<uint4 *>(dst)[g] =
+                make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
+          }
+        }
+      }
+    } else {
+      // per-column scale and bias of this chunk (warp-uniform addresses);
+      // issued before the TMEM load so the two latencies overlap
+      float sw[32];
+      uint32_t bw[16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int cg = col0 + 8 * g;
+        if (cg < p.N) {
+          const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg));
+          const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg) + 1);
+          sw[8 * g + 0] = w0.x; sw[8 * g + 1] = w0.y; sw[8 * g + 2] = w0.z; sw[8 * g + 3] = w0.w;
+          sw[8 * g + 4] = w1.x; sw[8 * g + 5] = w1.y; sw[8 * g + 6] = w1.z; sw[8 * g + 7] = w1.w;
+          if (p.bias != nullptr) {
+            const uint4 braw = __ldg(reinterpret_cast<const uint4 *>(p.bias + cg));
+            bw[4 * g + 0] = braw.x; bw[4 * g + 1] = braw.y;
+            bw[4 * g + 2] = braw.z; bw[4 * g + 3] = braw.w;
+          } else {
+            bw[4 * g + 0] = bw[4 * g + 1] = bw[4 * g + 2] = bw[4 * g + 3] = 0u;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sw[8 * g + i] = 0.0f;
+          bw[4 * g + 0] = bw[4 * g + 1] = bw[4 * g + 2] = bw[4 * g + 3] = 0u;
+        }
+      }
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(t_row + c, r);
+      tmem_ld_wait();
+      uint32_t packed[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float v0 = __int2float_rn(static_cast<int32_t>(r[2 * i]));
+        float v1 = __int2float_rn(static_cast<int32_t>(r[2 * i + 1]));
+        v0 = __fmul_rn(__fmul_rn(v0, sa), sw[2 * i]);
+        v1 = __fmul_rn(__fmul_rn(v1, sa), sw[2 * i + 1]);
+        if (p.bias != nullptr) {
+          v0 = __fadd_rn(v0, __uint_as_float(bw[i] << 16));
+          v1 = __fadd_rn(v1, __uint_as_float(bw[i] & 0xFFFF0000u));
+        }
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+        packed[i] = *reinterpret_cast<const uint32_t *>(&h);
+      }
+      // staging buffer of this chunk: free once the store issued two
+      // chunks ago has finished reading it
+      uint8_t *buf = stage_buf + (chunk_count & 1u) * kEpiBufBytes;
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+      // row `lane` = 64 bytes = four 16-byte pieces; 64-byte swizzle:
+      // piece j of row r sits at position j ^ ((r >> 1) & 3)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int pos = j ^ ((lane >> 1) & 3);
+        *reinterpret_cast<uint4 *>(buf + lane * 64 + pos * 16) =
+            make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmap_y, buf, col0, row0);
+        bulk_commit_group();
+      }
+      ++chunk_count;
+    }
+  }
+}
+
 template <int BN, int STAGES, bool RAW_OUT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_i8_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_a,
@@ -229,7 +327,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int e = warp - 2;            // 0..7
     const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31 = tile rows
     const int half = e >> 2;           // which half of the tile's columns
-    constexpr int kCols = BN / 2;      // columns per warp
     uint8_t *stage_buf = smem + L::kEpiOffset + e * 2 * kEpiBufBytes;
     uint32_t chunk_count = 0;          // TMA stores issued by this warp
     int acc = 0;
@@ -237,102 +334,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
       int mb, nb;
       gemm_tile_coords(t, p, mb, nb);
-      const int row0 = mb * kBM + quarter * 32;
-      const int row = row0 + lane;
-      const bool row_ok = row < p.M;
-      const float sa = row_ok ? __ldg(p.s_a + row) : 0.0f;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], acc_phase, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN + half * kCols);
-      // a warp whose 32 rows all lie past M has nothing to store
-      const int cols_here = row0 < p.M ? kCols : 0;
-#pragma unroll 1
-      for (int c = 0; c < cols_here; c += kEpiChunk) {
-        const int col0 = nb * BN + half * kCols + c;
-        if (col0 >= p.N) break;  // warp-uniform
-        if constexpr (RAW_OUT) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(t_row + c, r);
-          tmem_ld_wait();
-          if (row_ok) {
-            int32_t *dst = p.acc_out + static_cast<int64_t>(row) * p.N + col0;
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {
-              if (col0 + 4 * g < p.N) {
-                reinterpret_cast<uint4 *>(dst)[g] =
-                    make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]);
-              }
-            }
-          }
-        } else {
-          // per-column scale and bias of this chunk (warp-uniform addresses);
-          // issued before the TMEM load so the two latencies overlap
-          float sw[32];
-          uint32_t bw[16];
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int cg = col0 + 8 * g;
-            if (cg < p.N) {
-              const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg));
-              const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg) + 1);
-              sw[8 * g + 0] = w0.x; sw[8 * g + 1] = w0.y; sw[8 * g + 2] = w0.z; sw[8 * g + 3] = w0.w;
-              sw[8 * g + 4] = w1.x; sw[8 * g + 5] = w1.y; sw[8 * g + 6] = w1.z; sw[8 * g + 7] = w1.w;
-              if (p.bias != nullptr) {
-                const uint4 braw = __ldg(reinterpret_cast<const uint4 *>(p.bias + cg));
-                bw[4 * g + 0] = braw.x; bw[4 * g + 1] = braw.y;
-                bw[4 * g + 2] = braw.z; bw[4 * g + 3] = braw.w;
-              } else {
-                bw[4 * g + 0] = bw[4 * g + 1] = bw[4 * g + 2] = bw[4 * g + 3] = 0u;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) sw[8 * g + i] = 0.0f;
-              bw[4 * g + 0] = bw[4 * g + 1] = bw[4 * g + 2] = bw[4 * g + 3] = 0u;
-            }
-          }
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(t_row + c, r);
-          tmem_ld_wait();
-          uint32_t packed[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float v0 = __int2float_rn(static_cast<int32_t>(r[2 * i]));
-            float v1 = __int2float_rn(static_cast<int32_t>(r[2 * i + 1]));
-            v0 = __fmul_rn(__fmul_rn(v0, sa), sw[2 * i]);
-            v1 = __fmul_rn(__fmul_rn(v1, sa), sw[2 * i + 1]);
-            if (p.bias != nullptr) {
-              v0 = __fadd_rn(v0, __uint_as_float(bw[i] << 16));
-              v1 = __fadd_rn(v1, __uint_as_float(bw[i] & 0xFFFF0000u));
-            }
-            const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-            packed[i] = *reinterpret_cast<const uint32_t *>(&h);
-          }
-          // staging buffer of this chunk: free once the store issued two
-          // chunks ago has finished reading it
-          uint8_t *buf = stage_buf + (chunk_count & 1u) * kEpiBufBytes;
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
-          // row `lane` = 64 bytes = four 16-byte pieces; 64-byte swizzle:
-          // piece j of row r sits at position j ^ ((r >> 1) & 3)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int pos = j ^ ((lane >> 1) & 3);
-            *reinterpret_cast<uint4 *>(buf + lane * 64 + pos * 16) =
-                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmap_y, buf, col0, row0);
-            bulk_commit_group();
-          }
-          ++chunk_count;
-        }
-      }
+                             static_cast<uint32_t>(acc * BN + half * (BN / 2));
+      epilogue_warp_slice<BN / 2, RAW_OUT>(p, &tmap_y, t_row, mb * kBM + quarter * 32,
+                                           nb * BN + half * (BN / 2), stage_buf, chunk_count,
+                                           lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -352,6 +363,216 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------
+// CTA-pair variant (tcgen05 .cta_group::2): a cluster of two CTAs on two SMs
+// computes 256 x 256 output tiles.  CTA r of the pair loads rows
+// [128 r, 128 r + 128) of the tile's q block and rows [128 r, 128 r + 128) of
+// its Wq block (no multicast: each CTA loads its own halves), so a stage is
+// 32 KB per CTA instead of 48 KB and the ring is 6 deep; the leader CTA
+// (rank 0) issues M = 256, N = 256 MMAs that read both CTAs' shared memory
+// and accumulate into both CTAs' TMEM (CTA r holds rows 128 r .. 128 r + 127
+// of the tile, all 256 columns).  Both CTAs' TMA loads report to the
+// leader's "full" barrier; the leader's commits arrive on "empty" and
+// accumulator-"full" barriers in both CTAs; both CTAs' epilogue warps arrive
+// on the leader's accumulator-"empty" barrier.
+constexpr int kPairBN = 256;
+
+template <int STAGES>
+struct PairLayout {
+  static constexpr int kABytes = kBM * kBK;              // this CTA's 128 rows of q
+  static constexpr int kBBytes = (kPairBN / 2) * kBK;    // this CTA's 128 rows of Wq
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTileBytes = STAGES * kStageBytes;
+  static constexpr int kEpiOffset = kTileBytes;  // 1024-aligned
+  static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiBufBytes;
+  static constexpr int kBarOffset = kEpiOffset + kEpiBytes;
+  static constexpr int kBarBytes = (2 * STAGES + 5) * 8 + 8;
+  static constexpr int kSmemBytes = kBarOffset + kBarBytes + 1024;
+  static constexpr int kTmemCols = 2 * kPairBN;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+// Pair tile t -> (256-row block, 256-column block), banded like gemm_tile_coords.
+__device__ __forceinline__ void pair_tile_coords(int t, const GemmParams &p, int &mb, int &nb) {
+  gemm_tile_coords(t, p, mb, nb);  // p.num_m_blk counts 256-row blocks here
+}
+
+template <int STAGES, bool RAW_OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_i8_tcgen05_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                                const __grid_constant__ CUtensorMap tmap_b,
+                                const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+  using L = PairLayout<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBarOffset);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *drain = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader
+  const int pair_id = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);   // the leader's expect-tx arrival; bytes from both CTAs
+      mbar_init(&empty[s], 1);  // the leader's MMA commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * kEpiWarps);  // epilogue warps of both CTAs
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b);
+    if constexpr (!RAW_OUT) tma_prefetch_desc(&tmap_y);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, L::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialized, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int t = pair_id; ok && t < p.num_tiles; t += num_pairs) {
+        int mb, nb;
+        pair_tile_coords(t, p, mb, nb);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t *sa = smem + stage * L::kStageBytes;
+          uint8_t *sb = sa + L::kABytes;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::kStageBytes);
+          const uint32_t leader_full = map_to_cta(smem_addr(&full[stage]), 0);
+          tma_load_2d_pair(&tmap_a, leader_full, sa, kb * kBK, mb * 256 + static_cast<int>(rank) * 128);
+          tma_load_2d_pair(&tmap_b, leader_full, sb, kb * kBK, nb * kPairBN + static_cast<int>(rank) * 128);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // The leader's last commits still arrive on this CTA's "empty"
+      // barriers: wait for them before the CTA may leave (bounded).
+      const uint32_t n = issued < static_cast<uint32_t>(STAGES) ? issued : STAGES;
+      for (uint32_t i = issued - n; i < issued; ++i)
+        mbar_wait_drain(&empty[i % STAGES], (i / STAGES) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_i8(2 * kBM, kPairBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool any_mma = false;
+      for (int t = pair_id; ok && t < p.num_tiles; t += num_pairs) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPairBN);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_addr(smem + stage * L::kStageBytes);
+          const uint64_t adesc = smem_desc_k_sw128(sa);
+          const uint64_t bdesc = smem_desc_k_sw128(sa + L::kABytes);
+#pragma unroll
+          for (int k = 0; k < kBK / kMmaK; ++k)
+            mma_i8_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          any_mma = true;
+          mma_commit_pair(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[acc], 0x3);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok && any_mma) {
+        mma_commit_pair(drain, 0x1);
+        mbar_wait_drain(drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int e = warp - 2;
+    const int quarter = warp & 3;
+    const int half = e >> 2;
+    uint8_t *stage_buf = smem + L::kEpiOffset + e * 2 * kEpiBufBytes;
+    uint32_t chunk_count = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair_id; t < p.num_tiles; t += num_pairs) {
+      int mb, nb;
+      pair_tile_coords(t, p, mb, nb);
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&tfull[acc], acc_phase, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * kPairBN + half * (kPairBN / 2));
+      epilogue_warp_slice<kPairBN / 2, RAW_OUT>(
+          p, &tmap_y, t_row, mb * 256 + static_cast<int>(rank) * 128 + quarter * 32,
+          nb * kPairBN + half * (kPairBN / 2), stage_buf, chunk_count, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_cta(smem_addr(&tempty[acc]), 0));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if constexpr (!RAW_OUT) {
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
+    }
+  }
+
+  // Both CTAs finish (the leader's MMAs write the follower's TMEM, the
+  // follower's epilogue reads it) before either frees the pair's TMEM.
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, L::kTmemCols);
   }
 }
 
