@@ -363,7 +363,9 @@ def run_ours(args):
     layer.prepare_gemm_only()
     layer.i = 0
     gsteps = max(args.steps, 50)
-    tg = timed(layer.gemm_step, gsteps, warmup, dist, graph=True) / gsteps
+    gsampler = ClockSampler(dev.index if dev.index is not None else 0)
+    tg = timed(layer.gemm_step, gsteps, warmup, dist, gsampler, graph=True) / gsteps
+    gclk = gsampler.summary()
     layer.i = 0
     tq = timed(layer.quant_step, gsteps, warmup, dist, graph=True) / gsteps
     if gemv:
@@ -388,7 +390,13 @@ def run_ours(args):
                     "peak_basis": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
                                   f"nominal int8/bf16 ratio 2 (int8 ops counted as TOPS)",
                     "frac_of_nominal_4500": round(achieved / NOMINAL_INT8_TOPS, 4),
-                    "us_per_launch": round(tg * 1e6, 2)}
+                    "us_per_launch": round(tg * 1e6, 2),
+                    "sm_mhz_during_gemm": gclk.get("sm_mhz")}
+        if gclk.get("sm_mhz"):
+            # dense int8 tcgen05 rate: 16384 ops per SM per clock
+            clock_peak = 148 * 16384 * gclk["sm_mhz"] * 1e6 / 1e12
+            roofline["frac_of_clock_peak"] = round(achieved / clock_peak, 4)
+            roofline["clock_peak_tops"] = round(clock_peak, 1)
     quant_bytes = 3 * M * K + 4 * M
     extras = {
         "layer_us": round(sec_per_step * 1e6, 2),

@@ -209,22 +209,39 @@ int encode_bf16_store_map(CUtensorMap *map, const void *base, int64_t rows, int6
 
 // ---------------------------------------------------------------- launches
 
+// Launch with cudaLaunchKernelEx.  dependent = programmatic dependent launch:
+// the kernel may start before the preceding work on the stream completes and
+// must call griddepcontrol.wait before touching anything that work produces
+// (the GEMM kernels do, before their first q / s_a read and any store).
 template <typename... KArgs, typename... Args>
-int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-           Args... args) {
+int launch_ex(bool dependent, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+              cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = nullptr;
   cfg.numAttrs = 0;
+  if (dependent) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return W8A8_ERR_CUDA;
   }
   return W8A8_OK;
+}
+
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+           Args... args) {
+  return launch_ex(false, kernel, grid, block, smem, stream, args...);
 }
 
 // Raise a kernel's dynamic shared memory limit to `bytes`, once per device
@@ -320,8 +337,8 @@ int launch_gemm_t(const w8a8_plan &plan, const int8_t *q, const float *s_a, int6
   constexpr auto kernel = gemm_i8_tcgen05_kernel<BN, STAGES, RAW>;
   st = ensure_smem_limit<kernel>(L::kSmemBytes);
   if (st != W8A8_OK) return st;
-  return launch(kernel, dim3(plan.grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma, mb, my,
-                p);
+  return launch_ex(true, kernel, dim3(plan.grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma,
+                   mb, my, p);
 }
 
 template <bool RAW>
@@ -358,8 +375,8 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
   constexpr auto kernel = gemm_i8_tcgen05_pair_kernel<kGemmStagesPair, RAW>;
   st = ensure_smem_limit<kernel>(L::kSmemBytes);
   if (st != W8A8_OK) return st;
-  return launch(kernel, dim3(plan.grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma, mb, my,
-                p);
+  return launch_ex(true, kernel, dim3(plan.grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma,
+                   mb, my, p);
 }
 
 template <bool FUSED, bool RAW>

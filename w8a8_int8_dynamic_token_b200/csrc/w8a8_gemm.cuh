@@ -154,18 +154,20 @@ __device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const C
       uint32_t r[32];
       tmem_ld_32x32b_x32(t_row + c, r);
       tmem_ld_wait();
+      // two adjacent columns at a time in packed fp32: each lane of every
+      // packed operation is the same separately rounded operation as before
       uint32_t packed[16];
+      const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        float v0 = __int2float_rn(static_cast<int32_t>(r[2 * i]));
-        float v1 = __int2float_rn(static_cast<int32_t>(r[2 * i + 1]));
-        v0 = __fmul_rn(__fmul_rn(v0, sa), sw[2 * i]);
-        v1 = __fmul_rn(__fmul_rn(v1, sa), sw[2 * i + 1]);
-        if (p.bias != nullptr) {
-          v0 = __fadd_rn(v0, __uint_as_float(bw[i] << 16));
-          v1 = __fadd_rn(v1, __uint_as_float(bw[i] & 0xFFFF0000u));
-        }
-        const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+        float2 v = make_float2(__int2float_rn(static_cast<int32_t>(r[2 * i])),
+                               __int2float_rn(static_cast<int32_t>(r[2 * i + 1])));
+        v = mul2_rn(v, sa2);
+        v = mul2_rn(v, make_float2(sw[2 * i], sw[2 * i + 1]));
+        if (p.bias != nullptr)
+          v = add2_rn(v, make_float2(__uint_as_float(bw[i] << 16),
+                                     __uint_as_float(bw[i] & 0xFFFF0000u)));
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
         packed[i] = *reinterpret_cast<const uint32_t *>(&h);
       }
       // staging buffer of this chunk: free once the store issued two
@@ -244,6 +246,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       uint32_t issued = 0;
       bool ok = true;
+      // The weights do not depend on the preceding kernel: the first ring's
+      // worth of Wq loads is issued before waiting for it (programmatic
+      // dependent launch); q is loaded only after the wait.
+      int prefetched = 0;
+      if (static_cast<int>(blockIdx.x) < p.num_tiles) {
+        int mb0, nb0;
+        gemm_tile_coords(blockIdx.x, p, mb0, nb0);
+        prefetched = p.k_blocks < STAGES ? p.k_blocks : STAGES;
+        for (int kb = 0; kb < prefetched; ++kb) {
+          uint8_t *sb = smem + kb * L::kStageBytes + L::kABytes;
+          mbar_arrive_expect_tx(&full[kb], L::kStageBytes);
+          tma_load_2d(&tmap_b, &full[kb], sb, kb * kBK, nb0 * BN);
+        }
+      }
+      grid_dependency_wait();
       for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
         int mb, nb;
         gemm_tile_coords(t, p, mb, nb);
@@ -254,9 +271,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           uint8_t *sa = smem + stage * L::kStageBytes;
           uint8_t *sb = sa + L::kABytes;
-          mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+          if (prefetched > 0) {
+            --prefetched;  // this stage's barrier is armed and its Wq tile is in flight
+          } else {
+            mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
+            tma_load_2d(&tmap_b, &full[stage], sb, kb * kBK, nb * BN);
+          }
           tma_load_2d(&tmap_a, &full[stage], sa, kb * kBK, mb * kBM);
-          tma_load_2d(&tmap_b, &full[stage], sb, kb * kBK, nb * BN);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -331,6 +352,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t chunk_count = 0;          // TMA stores issued by this warp
     int acc = 0;
     uint32_t acc_phase = 0;
+    grid_dependency_wait();            // s_a comes from the preceding kernel
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
       int mb, nb;
       gemm_tile_coords(t, p, mb, nb);
@@ -455,6 +477,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       uint32_t issued = 0;
       bool ok = true;
+      // Wq loads of the first ring's worth of stages before waiting for the
+      // preceding kernel (programmatic dependent launch); q after the wait.
+      int prefetched = 0;
+      if (pair_id < p.num_tiles) {
+        int mb0, nb0;
+        pair_tile_coords(pair_id, p, mb0, nb0);
+        prefetched = p.k_blocks < STAGES ? p.k_blocks : STAGES;
+        for (int kb = 0; kb < prefetched; ++kb) {
+          uint8_t *sb = smem + kb * L::kStageBytes + L::kABytes;
+          if (rank == 0) mbar_arrive_expect_tx(&full[kb], 2 * L::kStageBytes);
+          tma_load_2d_pair(&tmap_b, map_to_cta(smem_addr(&full[kb]), 0), sb, kb * kBK,
+                           nb0 * kPairBN + static_cast<int>(rank) * 128);
+        }
+      }
+      grid_dependency_wait();
       for (int t = pair_id; ok && t < p.num_tiles; t += num_pairs) {
         int mb, nb;
         pair_tile_coords(t, p, mb, nb);
@@ -465,10 +502,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
           uint8_t *sa = smem + stage * L::kStageBytes;
           uint8_t *sb = sa + L::kABytes;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::kStageBytes);
           const uint32_t leader_full = map_to_cta(smem_addr(&full[stage]), 0);
+          if (prefetched > 0) {
+            --prefetched;  // armed and Wq in flight already
+          } else {
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::kStageBytes);
+            tma_load_2d_pair(&tmap_b, leader_full, sb, kb * kBK,
+                             nb * kPairBN + static_cast<int>(rank) * 128);
+          }
           tma_load_2d_pair(&tmap_a, leader_full, sa, kb * kBK, mb * 256 + static_cast<int>(rank) * 128);
-          tma_load_2d_pair(&tmap_b, leader_full, sb, kb * kBK, nb * kPairBN + static_cast<int>(rank) * 128);
           ++issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -539,6 +581,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t chunk_count = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
+    grid_dependency_wait();  // s_a comes from the preceding kernel
     for (int t = pair_id; t < p.num_tiles; t += num_pairs) {
       int mb, nb;
       pair_tile_coords(t, p, mb, nb);
