@@ -125,7 +125,7 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     if (!gemv_fits(M, K, max_smem)) return W8A8_ERR_UNSUPPORTED_SHAPE;
     const int64_t smem = M * K;
     int per_sm = static_cast<int>((max_smem) / (smem + 1024));
-    per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+    per_sm = per_sm < 1 ? 1 : (per_sm > 2 ? 2 : per_sm);  // one resident wave
     const int64_t rows_per_cta = kGemvWarps * kGemvRows;
     int64_t grid = cdiv(N, rows_per_cta);
     const int64_t cap = static_cast<int64_t>(sms) * per_sm;
@@ -282,15 +282,15 @@ int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q,
     V = cdiv(nvec, G);
   }
   if (V > kQuantMaxV) {  // rows longer than 256 x 12 x 8 = 24576 elements
-    return launch(quant_rows_long_kernel, dim3(static_cast<unsigned>(rows)), dim3(256), 0, stream,
-                  xp, K, ldx, q, s);
+    return launch_ex(true, quant_rows_long_kernel, dim3(static_cast<unsigned>(rows)), dim3(256), 0,
+                     stream, xp, K, ldx, q, s);
   }
   const int rows_per_block = 256 / G;
   const int64_t grid = cdiv(rows, rows_per_block);
   const int r32 = static_cast<int>(rows), k32 = static_cast<int>(K);
 #define W8A8_QUANT_CASE(VV)                                                                \
-  return launch(quant_rows_kernel<VV>, dim3(static_cast<unsigned>(grid)), dim3(256), 0,     \
-                stream, xp, r32, k32, ldx, q, s, G)
+  return launch_ex(true, quant_rows_kernel<VV>, dim3(static_cast<unsigned>(grid)), dim3(256), \
+                   0, stream, xp, r32, k32, ldx, q, s, G)
   switch (V) {
     case 1: W8A8_QUANT_CASE(1);
     case 2: W8A8_QUANT_CASE(2);
@@ -380,16 +380,16 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
 }
 
 template <bool FUSED, bool RAW>
-int launch_gemv_m(const w8a8_plan &plan, const GemvParams &p, int max_smem,
+int launch_gemv_m(const w8a8_plan &plan, const GemvParams &p, int max_smem, int sms,
                   cudaStream_t stream) {
+  (void)sms;
   const int smem = p.M * p.K;
-  (void)max_smem;
 #define W8A8_GEMV_CASE(MT)                                                              \
   {                                                                                     \
     constexpr auto kernel = gemv_i8_kernel<MT, FUSED, RAW>;                             \
     int st = ensure_smem_limit<kernel>(kGemvMaxSmem);                                   \
     if (st != W8A8_OK) return st;                                                       \
-    return launch(kernel, dim3(plan.grid), dim3(kGemvThreads), smem, stream, p);        \
+    return launch_ex(true, kernel, dim3(plan.grid), dim3(kGemvThreads), smem, stream, p); \
   }
   if (p.M <= 1) W8A8_GEMV_CASE(1)
   if (p.M <= 2) W8A8_GEMV_CASE(2)
@@ -470,8 +470,8 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
     p.y = static_cast<uint16_t *>(y);
     p.ldy = ldy;
     p.acc_out = acc;
-    return acc ? launch_gemv_m<false, true>(plan, p, d->max_smem_optin, stream)
-               : launch_gemv_m<false, false>(plan, p, d->max_smem_optin, stream);
+    return acc ? launch_gemv_m<false, true>(plan, p, d->max_smem_optin, d->sms, stream)
+               : launch_gemv_m<false, false>(plan, p, d->max_smem_optin, d->sms, stream);
   }
   if (plan.variant == W8A8_VARIANT_GEMM_PAIR) {
     return acc ? launch_gemm_pair<true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc, stream)
@@ -658,7 +658,7 @@ int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const in
     p.ldy = ldy;
     p.q_out = q_out;
     p.s_a_out = s_a_out;
-    return launch_gemv_m<true, false>(plan, p, d->max_smem_optin, stream);
+    return launch_gemv_m<true, false>(plan, p, d->max_smem_optin, d->sms, stream);
   }
 
   int8_t *q = q_out;

@@ -285,6 +285,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      grid_dependents_launch();  // all loads issued: the next kernel may start its prologue
       if (!ok) {
         // let the last loads land before the block's shared memory goes away
         const uint32_t n = issued < static_cast<uint32_t>(STAGES) ? issued : STAGES;
@@ -518,6 +519,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      grid_dependents_launch();  // all loads issued: the next kernel may start its prologue
       // The leader's last commits still arrive on this CTA's "empty"
       // barriers: wait for them before the CTA may leave (bounded).
       const uint32_t n = issued < static_cast<uint32_t>(STAGES) ? issued : STAGES;

@@ -11,7 +11,9 @@
 //      (unfused variant) every CTA copies the given q rows into shared memory;
 //   2. each warp walks pairs of weight rows, every lane holding 8 16-byte
 //      vectors of each row in flight (evict-first loads; the first pair's
-//      loads are issued before step 1 so the prologue hides under them),
+//      loads are issued before step 1 so the prologue hides under them, and
+//      before waiting on the preceding kernel when launched as a programmatic
+//      dependent),
 //      accumulating M int32 dot products with dp4a (exact: every partial sum
 //      is bounded by 127*127*K < 2^31);
 //   3. a warp reduction, then lane m writes
@@ -21,6 +23,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "w8a8_ptx.cuh"
 #include "w8a8_quant.cuh"
 
 namespace w8a8 {
@@ -96,9 +99,12 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_i8_kernel(const GemvParams 
   int pi = blockIdx.x * kGemvWarps + warp;
 
   // The weight stream is what this kernel waits on: start it before the
-  // activation prologue.
+  // activation prologue -- and, under programmatic dependent launch, before
+  // waiting for the preceding kernel (the weights do not depend on it; x, q
+  // and s_a may, so they are read only after the wait).
   uint4 wv[kGemvRows][kGemvVec];
   if (pi < npairs) gemv_load(p.wq, p.N, nvec16, pi * kGemvRows, 0, lane, wv);
+  grid_dependency_wait();
 
   // ---- 1. activation rows -> shared memory (int8) + scales
   if constexpr (FUSED) {
@@ -125,6 +131,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_i8_kernel(const GemvParams 
     if (tid < p.M) sas[tid] = __ldg(p.s_a + tid);
   }
   __syncthreads();
+  grid_dependents_launch();  // every CTA is resident; the next kernel may be scheduled
   if constexpr (FUSED) {
     if (blockIdx.x == 0) {
       if (p.q_out != nullptr) {

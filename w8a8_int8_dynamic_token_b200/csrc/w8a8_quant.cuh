@@ -133,6 +133,8 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const uint16_t *__
   const int tid = threadIdx.x;
   const int64_t nvec = K >> 3;
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * ldx);
+  grid_dependency_wait();  // see quant_rows_kernel
+  grid_dependents_launch();
   float m = 0.0f;
   for (int64_t vi = tid; vi < nvec; vi += 256) m = absmax_vec8(__ldg(xr + vi), m);
   uint32_t mb = warp_max_u32(__float_as_uint(m), 32);
@@ -176,12 +178,16 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t *__restr
   const int nvec = K >> 3;
 
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + (row_ok ? row : 0) * ldx);
+  // launched as a programmatic dependent: x may come from the preceding
+  // kernel, and q / s may still be read by it -- wait before either
+  grid_dependency_wait();
   uint4 v[V];
 #pragma unroll
   for (int j = 0; j < V; ++j) {
     const int vi = t + j * G;
     v[j] = (row_ok && vi < nvec) ? __ldcs(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
   }
+  grid_dependents_launch();  // the GEMM that follows may start its prologue
   float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
   for (int j = 0; j < V; ++j) {
