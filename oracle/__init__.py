@@ -54,6 +54,10 @@ def _load():
     lib.w8a8_oracle_epilogue.restype = ctypes.c_int
     lib.w8a8_oracle_linear.argtypes = [vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp]
     lib.w8a8_oracle_linear.restype = i64
+    lib.w8a8_oracle_pack_int32.argtypes = [vp, i64, i64, vp]
+    lib.w8a8_oracle_pack_int32.restype = None
+    lib.w8a8_oracle_unpack_int32.argtypes = [vp, i64, i64, vp]
+    lib.w8a8_oracle_unpack_int32.restype = None
     lib.w8a8_oracle_f32_to_bf16.argtypes = [ctypes.c_float]
     lib.w8a8_oracle_f32_to_bf16.restype = ctypes.c_uint16
     lib.w8a8_oracle_set_threads.argtypes = [ctypes.c_int]
@@ -176,6 +180,31 @@ def linear(x_bits: np.ndarray, wq: np.ndarray, s_w: np.ndarray, bias_bits=None) 
     if ov > 0:
         raise OverflowError(f"{ov} accumulators do not fit int32")
     return {"q": q, "s_a": s_a, "acc": acc, "y32": y32, "y": y}
+
+
+def pack_int32(wq: np.ndarray) -> np.ndarray:
+    """int8 [N, K] codes -> int32 [N, K/4] words: each code + 128 as a byte,
+    four consecutive codes per word, the first in the least significant byte
+    (the serialized weight storage; the order inside a word is this module's
+    reading of the pages)."""
+    wq = _as_c(wq, np.int8)
+    N, K = wq.shape
+    if K % 4:
+        raise ValueError("K must be a multiple of 4")
+    out = np.empty((N, K // 4), np.int32)
+    _load().w8a8_oracle_pack_int32(_ptr(wq), N, K, _ptr(out))
+    return out
+
+
+def unpack_int32(packed: np.ndarray, K: int) -> np.ndarray:
+    """int32 [N, K/4] words -> int8 [N, K] codes (inverse of pack_int32)."""
+    packed = _as_c(packed, np.int32)
+    N = packed.shape[0]
+    if packed.shape[1] * 4 != K:
+        raise ValueError("packed must be [N, K/4]")
+    out = np.empty((N, K), np.int8)
+    _load().w8a8_oracle_unpack_int32(_ptr(packed), N, K, _ptr(out))
+    return out
 
 
 def library_path() -> str:

@@ -184,6 +184,42 @@ int64_t w8a8_oracle_linear(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
     return ov;
 }
 
+/* ---- packed int32 weight storage ----------------------------------------- */
+
+/*
+ * The serialized form of an int8 weight: each code stored as an unsigned byte
+ * biased by 128, four bytes per int32 word ("Qwen-Image-2.1: TE AutoRound-AWQ
+ * on GPU + all-resident single-3090 stack", the artifact description of the
+ * quantized transformer built with compressed-tensors' pack_to_int32).  The
+ * pages fix the bias and the four-per-word ratio; the order inside a word is
+ * taken as consecutive codes along K, the first in the least significant
+ * byte.  packed is int32 [N][K/4] (K a multiple of 4), Wq int8 [N][K].
+ */
+void w8a8_oracle_pack_int32(const int8_t *wq, int64_t N, int64_t K, int32_t *packed)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < K / 4; ++g) {
+            uint32_t word = 0;
+            for (int j = 0; j < 4; ++j) {
+                uint32_t biased = (uint32_t)((int32_t)wq[n * K + 4 * g + j] + 128);
+                word |= biased << (8 * j);
+            }
+            packed[n * (K / 4) + g] = (int32_t)word;
+        }
+    }
+}
+
+void w8a8_oracle_unpack_int32(const int32_t *packed, int64_t N, int64_t K, int8_t *wq)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            uint32_t word = (uint32_t)packed[n * (K / 4) + k / 4];
+            int32_t biased = (int32_t)((word >> (8 * (k % 4))) & 0xFFu);
+            wq[n * K + k] = (int8_t)(biased - 128);
+        }
+    }
+}
+
 /* ---- helpers for the Python side ---------------------------------------- */
 
 uint16_t w8a8_oracle_f32_to_bf16(float f) { return f32_to_bf16_rne(f); }

@@ -384,3 +384,54 @@ def test_planted_wrong_divisor_or_rounding_fails_pin():
     q, s = oracle.quant_rows(x)
     assert q.tolist() != q_away.tolist()
     assert q.tolist() == [[127, 0, 2, -2, 64]]
+
+
+# --------------------------------------------------------------------------
+# Packed int32 weight storage: codes biased by 128, four per int32 word
+# ("Qwen-Image-2.1: TE AutoRound-AWQ on GPU + all-resident single-3090 stack",
+# the quantized-transformer artifact built with pack_to_int32).  The order
+# inside a word is a reading: consecutive codes along K, first code in the
+# least significant byte.
+# --------------------------------------------------------------------------
+
+def test_pack_int32_worked_example():
+    # codes -128, -1, 0, 127 -> biased bytes 0x00, 0x7F, 0x80, 0xFF, first
+    # byte least significant -> 0xFF807F00
+    p = oracle.pack_int32(np.array([[-128, -1, 0, 127]], np.int8))
+    assert p.shape == (1, 1) and (int(p[0, 0]) & 0xFFFFFFFF) == 0xFF807F00
+    assert oracle.unpack_int32(p, 4).tolist() == [[-128, -1, 0, 127]]
+
+
+def test_pack_int32_every_code_at_every_byte_position():
+    codes = np.arange(-128, 128, dtype=np.int16).astype(np.int8)
+    for j in range(4):
+        wq = np.zeros((256, 8), np.int8)
+        wq[:, j] = codes
+        wq[:, 4 + (3 - j)] = codes[::-1]
+        p = oracle.pack_int32(wq)
+        # the word's bytes in memory order (little-endian host) are the codes + 128
+        assert np.array_equal(p.view(np.uint8).reshape(256, 8),
+                              (wq.astype(np.int16) + 128).astype(np.uint8))
+        shifted = (p[:, 0].astype(np.int64) & 0xFFFFFFFF) >> (8 * j) & 0xFF
+        assert np.array_equal(shifted, codes.astype(np.int64) + 128)
+        assert np.array_equal(oracle.unpack_int32(p, 8), wq)
+
+
+def test_pack_int32_round_trip_random():
+    wq = np.random.default_rng(4).integers(-128, 128, size=(37, 64), dtype=np.int8)
+    p = oracle.pack_int32(wq)
+    assert p.shape == (37, 16)
+    assert np.array_equal(oracle.unpack_int32(p, 64), wq)
+
+
+def test_planted_packing_mistakes_fail_pin():
+    wq = np.array([[-128, -1, 0, 127]], np.int8)
+    # most significant byte first
+    be = np.array([[int.from_bytes(bytes((wq.astype(np.int16) + 128).astype(np.uint8)[0]), "big")]],
+                  np.uint32).view(np.int32)
+    # bias by -128 (two's complement byte) instead of +128
+    raw = np.array([[int.from_bytes(bytes(wq.view(np.uint8)[0]), "little")]],
+                   np.uint32).view(np.int32)
+    good = oracle.pack_int32(wq)
+    assert not np.array_equal(be, good) and not np.array_equal(raw, good)
+    assert oracle.unpack_int32(be, 4).tolist() != wq.tolist()
