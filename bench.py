@@ -212,7 +212,8 @@ class Layer:
     def gemm_step(self):
         s = self.sets[self.i]
         self.i = (self.i + 1) % len(self.sets)
-        self.w8a8.linear(s["q"], s["s_a"], s["Wq"], s["s_w"], s["b"], out=s["y"])
+        self.w8a8.linear(s["q"], s["s_a"], s["Wq"], s["s_w"], s["b"], out=s["y"],
+                         workspace=s["ws"])
 
     def quant_step(self):
         s = self.sets[self.i]
@@ -502,7 +503,38 @@ def extra_components(args, dev, dist, peaks, world):
                            "frac_of_nominal_4500": round(ops / t / 1e12 / NOMINAL_INT8_TOPS, 4)}
         del layers, up, down
         torch.cuda.empty_cache()
+        out["dit_block"] = dit_block_component(dev, dist, max(10, steps // 4))
     return out
+
+
+def dit_block_component(dev, dist, steps):
+    """One DiT block's quantized linears at CFG batch 2, launched back to back
+    on one stream (each call's kernels are programmatic dependents of the
+    previous call's): eager launches and a CUDA graph of the block."""
+    layers = [Layer(c, dev) for c in synth.DIT_BLOCK]
+
+    def block():
+        for L in layers:
+            L.step()
+
+    t = timed(block, steps, 3, dist) / steps
+    for L in layers:
+        L.i = 0
+    t_graph = timed(block, steps, 3, dist, graph=True) / steps
+    per_layer = {}
+    for L in layers:
+        L.i = 0
+        per_layer[L.case.name] = round(timed(L.step, steps, 3, dist, graph=True) / steps * 1e6, 2)
+    ops = sum(c.ops for c in synth.DIT_BLOCK)
+    res = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
+           "us_graph": round(t_graph * 1e6, 2), "TOPS_graph": round(ops / t_graph / 1e12, 1),
+           "frac_of_nominal_4500_graph": round(ops / t_graph / 1e12 / NOMINAL_INT8_TOPS, 4),
+           "layers_us_graph_alone": per_layer,
+           "calls": [f"{c.name} M={c.M} K={c.K} N={c.N}" for c in synth.DIT_BLOCK],
+           "gpu_launches_per_block": sum(L.launches_per_step for L in layers)}
+    del layers
+    torch.cuda.empty_cache()
+    return res
 
 
 # ----------------------------------------------------------------------------- reference arm

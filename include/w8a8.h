@@ -92,7 +92,13 @@ typedef struct {
     int32_t tile_n;        /* columns of y per tile (GEMM) or 0 */
     int32_t num_tiles;     /* GEMM tiles, or GEMV output rows of W */
     int32_t grid;          /* CTAs launched */
-    int32_t waves_x100;    /* 100 * num_tiles / grid (GEMM), else 0 */
+    int32_t waves_x100;    /* tile rounds per CTA (pair) x 100, counting the
+                              K-split tail as its share of a round (GEMM), else 0 */
+    int32_t split_tiles;   /* GEMM_PAIR: the last split_tiles tiles (one to two
+                              waves) are shared out along K among all pairs;
+                              0 = none */
+    int32_t split_kblocks_per_pair; /* GEMM_PAIR with split_tiles > 0: 128-deep
+                              k-blocks of that region per pair, else 0 */
 } w8a8_plan;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -108,6 +114,23 @@ W8A8_API int w8a8_quantize_weights(const void *W_bf16, int64_t N, int64_t K, int
                           int8_t *Wq, float *s_w, w8a8_stream_t stream);
 
 /*
+ * Weight loading from packed int32 storage, run once per layer at load time
+ * (the serialized checkpoint form: "Qwen-Image-2.1: TE AutoRound-AWQ on GPU +
+ * all-resident single-3090 stack", the quantized-transformer artifact built
+ * with pack_to_int32 -- each int8 code stored as an unsigned byte biased by
+ * 128, four per int32 word).  packed int32 [N, K/4] dense: word g of row n
+ * holds the codes of columns 4g .. 4g+3, column 4g in the least significant
+ * byte -> Wq int8 [N,K] dense, Wq[n,k] = byte - 128.  The per-channel scales
+ * s_w are stored beside the packed codes and are used as they are.
+ * A code of -128 (byte 0) is passed through; with such codes the GEMM is
+ * exact for K <= 132104 (127 * 128 * K < 2^31).
+ * Preconditions as for w8a8_quantize_weights (K % 16 == 0, both pointers
+ * 16-byte aligned).
+ */
+W8A8_API int w8a8_unpack_int32_weights(const int32_t *packed, int64_t N, int64_t K, int8_t *Wq,
+                                       w8a8_stream_t stream);
+
+/*
  * Per-token dynamic activation quantization.
  * x bf16 [M,K] (row stride ldx) -> q int8 [M,K] dense, s_a fp32 [M].
  */
@@ -115,9 +138,11 @@ W8A8_API int w8a8_quant_act(const void *x_bf16, int64_t M, int64_t K, int64_t ld
                    int8_t *q, float *s_a, w8a8_stream_t stream);
 
 /*
- * Scratch bytes w8a8_linear_fused needs for (M, N, K) (the int8 activations
- * and their scales when they are not returned through q_out / s_a_out).
- * w8a8_linear needs none; it accepts workspace = NULL, ws_bytes = 0.
+ * Scratch bytes for (M, N, K) on a 148-SM B200: w8a8_linear_fused's int8
+ * activations and their scales, plus, when the plan shares its last tiles
+ * out along K (w8a8_plan.split_tiles > 0), the int32 partial sums and arrival
+ * counters of that region.  A workspace too small for the K-split region
+ * still works: the layer then runs without the split (slower tail wave).
  */
 W8A8_API int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes);
 
@@ -127,7 +152,13 @@ W8A8_API int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes)
  * bias bf16 [N] or NULL -> y bf16 [M,N] (row stride ldy).
  * acc_debug: NULL, or int32 [M,N] dense; when given, the raw int32
  * accumulators are written there INSTEAD of y (y may then be NULL).
- * workspace / ws_bytes: unused (may be NULL / 0).
+ * workspace / ws_bytes: optional (NULL / 0 allowed).  With at least
+ * w8a8_workspace_size(M,N,K) bytes (16-byte aligned) the pair kernel's K-split
+ * tail is used.  Its contents need no initialization (arrival counters carry
+ * a per-launch tag and are reset by the kernel); the workspace must not be in
+ * use by other work while the call runs.  After a launch that reported
+ * W8A8_ERR_DEVICE_TIMEOUT, replaying a captured graph of it on the same
+ * workspace is outside the contract.
  */
 W8A8_API int w8a8_linear(const int8_t *q, const float *s_a, int64_t M, int64_t K,
                 const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,
@@ -135,19 +166,22 @@ W8A8_API int w8a8_linear(const int8_t *q, const float *s_a, int64_t M, int64_t K
                 void *workspace, size_t ws_bytes, w8a8_stream_t stream);
 
 /* w8a8_linear with an explicit kernel variant (AUTO = the selector's choice).
- * GEMV requires M <= 16. */
+ * GEMV requires M <= 16.  workspace as in w8a8_linear (GEMM_PAIR uses it for
+ * the K-split tail when large enough; NULL runs the pair kernel unsplit). */
 W8A8_API int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K,
                    const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,
                    void *y_bf16, int64_t ldy, int32_t *acc_debug_or_null,
-                   int variant, w8a8_stream_t stream);
+                   int variant, void *workspace, size_t ws_bytes, w8a8_stream_t stream);
 
 /*
  * The whole layer from bf16 activations: quantize x per token, then the int8
  * GEMM with the fused epilogue.  x bf16 [M,K] (row stride ldx) -> y bf16 [M,N].
  * q_out / s_a_out: NULL, or int8 [M,K] dense / fp32 [M] to receive the
  * intermediates (then they are used instead of workspace).
- * workspace: at least w8a8_workspace_size(M,N,K) bytes unless both q_out and
- * s_a_out are given; 256-byte alignment is recommended.
+ * workspace: w8a8_workspace_size(M,N,K) bytes, 16-byte aligned (256
+ * recommended).  Required: the bytes for q and s_a, unless both q_out and
+ * s_a_out are given; the rest (the K-split region) is optional, see
+ * w8a8_workspace_size.
  */
 W8A8_API int w8a8_linear_fused(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
                       const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,

@@ -116,6 +116,19 @@ FFN_DOWN = LayerCase("ffn_down", 4352, 12288, 3072, "gelu", 0)
 ADALN_M1 = LayerCase("adaln_m1", 1, 3072, 18432, "normal", 0)
 ADALN_M2 = LayerCase("adaln_m2", 2, 3072, 18432, "normal", 0)
 
+# One DiT block's quantized linears at CFG batch 2 (the conditional and
+# unconditional branches batched: M = 2 x 4352 tokens): the fused q|k|v
+# projection, the attention output projection, the fused FFN proj|gate
+# projection (two 3072 -> 12288 linears on the same input), the FFN output
+# projection, and the AdaLN modulation projection as a GEMV at M = 2.
+DIT_BLOCK = (
+    LayerCase("blk_qkv", 8704, 3072, 9216, "studentt", 10),
+    LayerCase("blk_to_out", 8704, 3072, 3072, "studentt", 11),
+    LayerCase("blk_proj_gate", 8704, 3072, 24576, "studentt", 12),
+    LayerCase("blk_ffn_out", 8704, 12288, 3072, "gelu", 13),
+    LayerCase("blk_adaln", 2, 3072, 18432, "normal", 14),
+)
+
 SWEEP_M = (1, 16, 17, 256, 1024, 4352, 8704, 16384)
 SWEEP_KN = ((3072, 9216), (3072, 3072), (3072, 12288), (12288, 3072))
 SWEEP_SEEDS = (0, 1, 2, 3)

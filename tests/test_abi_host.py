@@ -71,7 +71,7 @@ def test_null_and_misaligned_pointers():
         B.W8A8_ERR_MISALIGNED
     assert B.w8a8_linear(P, P, 4, 16, P, P, None, 12, P, 12, None, None, 0, None) == \
         B.W8A8_ERR_UNSUPPORTED_SHAPE   # N % 8
-    assert B.w8a8_linear_ex(P, P, 4, 16, P, P, None, 8, P, 8, None, 9, None) == \
+    assert B.w8a8_linear_ex(P, P, 4, 16, P, P, None, 8, P, 8, None, 9, None, 0, None) == \
         B.W8A8_ERR_INVALID_ARG         # unknown variant
 
 
@@ -128,6 +128,83 @@ def test_workspace_size_covers_q_and_scales():
     M, N, K = 4352, 9216, 3072
     n = w8a8.workspace_size(M, N, K)
     assert n >= M * K + 4 * M and n % 256 == 0
+
+
+# The pair kernel's schedule: whole tiles in full waves, then the last one to
+# two waves' tiles shared out along K in equal runs of k-blocks per pair.  A
+# model of the device-side partition (work items, contributor counts, partial
+# slots) checks that every (tile, k-block) is computed exactly once and that
+# the partial-sum slots of different contributions never collide.
+def _pair_items(tiles, split_tiles, per, kb, pairs, pair):
+    tile0 = tiles - split_tiles
+    items = [(t, 0, kb, 1, 0) for t in range(pair, tile0, pairs)]
+    if split_tiles:
+        units = split_tiles * kb
+        u0, u1 = pair * per, min(pair * per + per, units)
+        t = u0 // kb if u0 < u1 else None
+        while t is not None and t * kb < u1:
+            first, last = (t * kb) // per, ((t + 1) * kb - 1) // per
+            items.append((tile0 + t, max(u0 - t * kb, 0), min(u1 - t * kb, kb),
+                          last - first + 1, pair - first))
+            t += 1
+    return items
+
+
+SPLIT_SHAPES = [(4352, 9216, 3072), (4352, 12288, 3072), (4352, 3072, 12288), (512, 1024, 12288),
+                (640, 768, 1024), (200, 136, 12288), (1280, 4096, 1024), (2560, 8192, 512),
+                (8704, 9216, 3072), (16384, 3072, 12288), (512, 9472, 3072), (8704, 3072, 12288),
+                (600, 2056, 12288), (768, 1024, 133120)]
+
+
+@pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
+def test_pair_k_split_partition(M, N, K):
+    p = w8a8.select(M, N, K, variant=B.VARIANT_GEMM_PAIR)
+    tiles, pairs, kb = p["num_tiles"], p["grid"] // 2, -(-K // 128)
+    st, per = p["split_tiles"], p["split_kblocks_per_pair"]
+    if tiles % 74 == 0:
+        assert st == 0
+    if st:
+        assert per >= 24 and per * pairs >= st * kb
+        assert st <= tiles and (tiles - st) % pairs == 0 and st < 2 * pairs
+    covered = {}
+    slots = set()
+    for pair in range(pairs):
+        for t, b, e, nparts, part in _pair_items(tiles, st, per, kb, pairs, pair):
+            assert 0 <= b < e <= kb and 0 <= part < nparts
+            for k in range(b, e):
+                assert (t, k) not in covered
+                covered[(t, k)] = pair
+            if nparts > 1:
+                slot = (t - (tiles - st)) + pair
+                assert slot not in slots and slot < st + pairs - 1
+                slots.add(slot)
+    assert len(covered) == tiles * kb
+    # contributor counts agree with who actually covers each tile
+    for t in range(tiles - st, tiles):
+        owners = sorted({covered[(t, k)] for k in range(kb)})
+        assert owners == list(range(owners[0], owners[-1] + 1))
+
+
+def test_pair_k_split_plans():
+    # 408 tiles of 96 k-blocks: 4 full waves whole, 112 tiles shared out at
+    # 146 k-blocks per pair instead of a 6th wave of 96 (saves 46 >= 24)
+    p = w8a8.select(8704, 3072, 12288)
+    assert p["variant_name"] == "gemm_pair"
+    assert p["split_tiles"] == 408 - 4 * 74 and p["split_kblocks_per_pair"] == -(-112 * 96 // 74)
+    assert p["waves_x100"] == 400 + -(-100 * 146 // 96)
+    # short tiles: shared-out pieces would be epilogue-bound -> no split
+    for M, N, K in ((4352, 9216, 3072), (4352, 12288, 3072), (8704, 3072, 3072)):
+        assert w8a8.select(M, N, K)["split_tiles"] == 0
+    # a tail that is already three quarters full: the split saves too little
+    assert w8a8.select(4352, 3072, 12288)["split_tiles"] == 0
+    # under one wave with long K: shared out entirely in pieces of >= 24 k-blocks
+    p = w8a8.select(512, 1024, 12288, variant=B.VARIANT_GEMM_PAIR)
+    assert p["split_tiles"] == 8 and p["split_kblocks_per_pair"] == 24
+    p = w8a8.select(512, 9472, 3072, variant=B.VARIANT_GEMM_PAIR)   # exactly one wave
+    assert p["split_tiles"] == 0 and p["num_tiles"] == 74
+    # the workspace covers the K-split region: counters + (split + pairs - 1) slots of 256 KiB
+    n = w8a8.workspace_size(8704, 3072, 12288)
+    assert n >= 8704 * 12288 + 4 * 8704 + (112 + 73) * 256 * 1024
 
 
 @pytest.mark.parametrize("M", [17, 100, 4352, 16384])

@@ -349,3 +349,176 @@ def test_errors_are_returned_not_raised_in_c():
     with pytest.raises(w8a8.W8A8Error) as e:
         w8a8.quant_act(x)
     assert e.value.status == B.W8A8_ERR_UNSUPPORTED_SHAPE
+
+
+# ----------------------------------------------------------------- chained calls
+
+def test_chained_layers_share_buffers_under_dependent_launch():
+    """Consecutive layer calls are launched as programmatic dependents: each
+    kernel starts before the previous one finishes and waits for it before
+    touching its data.  A chain whose every input is the previous output, with
+    one workspace reused by every call and GEMV and GEMM layers interleaved,
+    must equal the oracle run step by step."""
+    K = 1024
+    dims = [(384, K), (2, K), (300, K), (1, K), (384, K)]   # (M, N=K) per step: GEMM/GEMV mix
+    rng_seed = 21
+    ws = torch.empty((w8a8.workspace_size(384, K, K) + 256,), dtype=torch.uint8, device="cuda")
+    x_bits = synth.make_x(384, K, "studentt", rng_seed)
+    weights = []
+    for i in range(len(dims)):
+        w = synth.make_w(K, K, rng_seed + i)
+        wq, sw = oracle.quantize_weights(w)
+        weights.append((wq, sw, synth.make_bias(K, rng_seed + i)))
+    # GPU: one stream, no synchronization between the calls
+    cur = to_dev(x_bits)
+    outs = []
+    for (M, _), (wq, sw, b) in zip(dims, weights):
+        y = w8a8.linear_fused(cur[:M], torch.from_numpy(wq).cuda(), torch.from_numpy(sw).cuda(),
+                              to_dev(b), workspace=ws)
+        outs.append(y)
+        nxt = torch.zeros((384, K), dtype=torch.bfloat16, device="cuda")
+        nxt[:M] = y
+        cur = nxt
+    torch.cuda.synchronize()
+    # oracle, step by step
+    ref_in = x_bits
+    for step, ((M, _), (wq, sw, b), y) in enumerate(zip(dims, weights, outs)):
+        r = oracle.linear(np.ascontiguousarray(ref_in[:M]), wq, sw, b)
+        assert check_y(bits_of(y), r["y"], r["y32"], f"chain step {step}") == 0
+        nxt = np.zeros((384, K), np.uint16)
+        nxt[:M] = r["y"]
+        ref_in = nxt
+
+
+def test_back_to_back_calls_reuse_one_workspace():
+    """Many fused calls on one workspace, no synchronization in between: the
+    quantization of call i+1 overwrites q / s_a that the GEMM of call i reads,
+    and must wait for it."""
+    M, N, K = 640, 1024, 3072
+    ws = torch.empty((w8a8.workspace_size(M, N, K),), dtype=torch.uint8, device="cuda")
+    w = synth.make_w(N, K, 31)
+    wq, sw = oracle.quantize_weights(w)
+    b = synth.make_bias(N, 31)
+    Wq, s_w, bd = torch.from_numpy(wq).cuda(), torch.from_numpy(sw).cuda(), to_dev(b)
+    xs = [synth.make_x(M, K, "studentt", 40 + i) for i in range(4)]
+    xs_dev = [to_dev(x) for x in xs]
+    outs = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in xs]
+    torch.cuda.synchronize()
+    for xd, o in zip(xs_dev, outs):   # nothing but these calls between the launches
+        w8a8.linear_fused(xd, Wq, s_w, bd, out=o, workspace=ws)
+    ys = outs
+    torch.cuda.synchronize()
+    for i, (x, y) in enumerate(zip(xs, ys)):
+        rows = sample_rows(M, seed=i, n_random=32)
+        r = oracle.linear(np.ascontiguousarray(x[rows]), wq, sw, b)
+        assert check_y(bits_of(y)[rows], r["y"], r["y32"], f"call {i}") == 0
+
+
+# ----------------------------------------------------------------- K-split tail
+
+# (M, N, K): under one wave, every tile shared by four pairs (512 x 1024 x
+# 12288), ragged edges in M and N with tiles shared by two or three pairs
+# (600 x 2056 x 12288), four full waves of whole tiles and then 112 tiles
+# shared out at 146 k-blocks per pair (8704 x 3072 x 12288).
+SPLIT_CASES = [(512, 1024, 12288), (600, 2056, 12288), (8704, 3072, 12288)]
+
+
+@pytest.mark.parametrize("M,N,K", SPLIT_CASES)
+def test_pair_k_split_matches_unsplit_and_oracle(M, N, K):
+    """The pair kernel with its last tiles shared out along K (partial int32
+    sums, last-arriver reduction) against the same kernel unsplit -- raw
+    accumulators and y, in full -- and against the oracle on sampled rows."""
+    plan = w8a8.select(M, N, K, variant=B.VARIANT_GEMM_PAIR)
+    assert plan["split_tiles"] > 0
+    rng = np.random.default_rng(M + N + K)
+    q = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
+    wq = rng.integers(-127, 128, size=(N, K), dtype=np.int8)
+    s_a = (rng.random(M, dtype=np.float32) * 0.05 + 1e-3).astype(np.float32)
+    s_w = (rng.random(N, dtype=np.float32) * 0.002 + 1e-4).astype(np.float32)
+    b = synth.make_bias(N, seed=5)
+    args = (torch.from_numpy(q).cuda(), torch.from_numpy(s_a).cuda(), torch.from_numpy(wq).cuda(),
+            torch.from_numpy(s_w).cuda(), to_dev(b))
+    acc_split = w8a8.linear(*args, acc_debug=True, variant=B.VARIANT_GEMM_PAIR)
+    acc_plain = w8a8.linear(*args, acc_debug=True, variant=B.VARIANT_GEMM_PAIR, split=False)
+    y_split = w8a8.linear(*args, variant=B.VARIANT_GEMM_PAIR)
+    y_plain = w8a8.linear(*args, variant=B.VARIANT_GEMM_PAIR, split=False)
+    torch.cuda.synchronize()
+    assert torch.equal(acc_split, acc_plain)
+    assert torch.equal(y_split, y_plain)
+    rows = sample_rows(M, seed=7, n_random=24, tile=256)
+    ref = oracle.gemm_i32(q[rows], wq)
+    assert np.array_equal(acc_split.cpu().numpy()[rows], ref)
+    y32, y_ref = oracle.epilogue(ref, s_a[rows], s_w, b)
+    assert check_y(bits_of(y_split)[rows], y_ref, y32, "k-split") == 0
+
+
+def test_pair_k_split_repeated_calls_on_one_workspace():
+    """Back-to-back split launches on one workspace: each call's counters are
+    cleared before its GEMM and no call reads another's partial sums."""
+    M, N, K = 512, 1024, 12288
+    assert w8a8.select(M, N, K, variant=B.VARIANT_GEMM_PAIR)["split_tiles"] > 0
+    rng = np.random.default_rng(99)
+    wq = rng.integers(-127, 128, size=(N, K), dtype=np.int8)
+    Wq = torch.from_numpy(wq).cuda()
+    ones_n = torch.ones(N, device="cuda")
+    ws = torch.empty((w8a8.workspace_size(M, N, K),), dtype=torch.uint8, device="cuda")
+    qs = [rng.integers(-127, 128, size=(M, K), dtype=np.int8) for _ in range(3)]
+    accs = [w8a8.linear(torch.from_numpy(q).cuda(), torch.ones(M, device="cuda"), Wq, ones_n,
+                        acc_debug=True, variant=B.VARIANT_GEMM_PAIR, workspace=ws) for q in qs]
+    torch.cuda.synchronize()
+    for i, (q, acc) in enumerate(zip(qs, accs)):
+        rows = sample_rows(M, seed=i, n_random=16, tile=256)
+        assert np.array_equal(acc.cpu().numpy()[rows], oracle.gemm_i32(q[rows], wq)), i
+
+
+# ----------------------------------------------------------------- packed weights
+
+@pytest.mark.parametrize("N,K", [(8, 16), (264, 3072), (18432, 3072), (3072, 12288)])
+def test_unpack_int32_weights_bitexact(N, K):
+    """Packed int32 storage (written by the oracle's packer) -> int8 codes on
+    the GPU, byte-equal to the oracle's unpacking; every code including -128."""
+    rng = np.random.default_rng(N + K)
+    wq = rng.integers(-128, 128, size=(N, K), dtype=np.int8)
+    wq[0, :min(K, 256)] = np.arange(-128, 128, dtype=np.int16).astype(np.int8)[:min(K, 256)]
+    packed = oracle.pack_int32(wq)
+    got = w8a8.unpack_int32_weights(torch.from_numpy(packed).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(got.cpu().numpy(), oracle.unpack_int32(packed, K))
+
+
+def test_unpacked_weights_drive_the_layer():
+    """A layer whose weights come from packed storage equals the layer with
+    the oracle's codes (the scales are stored beside the codes)."""
+    M, N, K = 300, 520, 3072
+    x, w, b = synth.make_x(M, K, "studentt", 8), synth.make_w(N, K, 8), synth.make_bias(N, 8)
+    wq, sw = oracle.quantize_weights(w)
+    Wq = w8a8.unpack_int32_weights(torch.from_numpy(oracle.pack_int32(wq)).cuda())
+    y = w8a8.linear_fused(to_dev(x), Wq, torch.from_numpy(sw).cuda(), to_dev(b))
+    torch.cuda.synchronize()
+    r = oracle.linear(x, wq, sw, b)
+    assert check_y(bits_of(y), r["y"], r["y32"], "packed weights") == 0
+
+
+# ----------------------------------------------------------------- DiT block
+
+def test_dit_block_linears_back_to_back():
+    """One DiT block's linear set at CFG batch 2 (fused q|k|v, to_out, fused
+    proj|gate, FFN out, AdaLN GEMV), launched back to back on one stream with
+    one shared workspace; every output against the oracle on sampled rows."""
+    cases = synth.DIT_BLOCK
+    ws = torch.empty((max(w8a8.workspace_size(c.M, c.N, c.K) for c in cases),),
+                     dtype=torch.uint8, device="cuda")
+    host, outs = [], []
+    for c in cases:
+        x, b = c.x(), c.b()
+        wq, sw = oracle.quantize_weights(c.w())
+        host.append((x, wq, sw, b))
+        outs.append((to_dev(x), torch.from_numpy(wq).cuda(), torch.from_numpy(sw).cuda(),
+                     to_dev(b)))
+    torch.cuda.synchronize()
+    ys = [w8a8.linear_fused(xd, Wq, s_w, bd, workspace=ws) for xd, Wq, s_w, bd in outs]
+    torch.cuda.synchronize()
+    for c, (x, wq, sw, b), y in zip(cases, host, ys):
+        rows = sample_rows(c.M, seed=c.seed, n_random=32, tile=256)
+        r = oracle.linear(np.ascontiguousarray(x[rows]), wq, sw, b)
+        assert check_y(bits_of(y)[rows], r["y"], r["y32"], c.name) == 0

@@ -9,5 +9,6 @@ dequantization/bias epilogue producing bf16.  The kernels live in
 from .binding import (  # noqa: F401
     LIB_PATH, VARIANT_AUTO, VARIANT_GEMM_BN128, VARIANT_GEMM_BN256, VARIANT_GEMM_PAIR, VARIANT_GEMV,
     W8A8Error, last_device_error, lib, linear, linear_fused, linear_fused_host, quant_act,
-    quantize_weights, select, selftest_bounded_wait, status_string, version, workspace_size,
+    quantize_weights, select, selftest_bounded_wait, status_string, unpack_int32_weights, version,
+    workspace_size,
 )

@@ -49,7 +49,8 @@ class W8A8Error(RuntimeError):
 class Plan(ctypes.Structure):
     _fields_ = [("variant", ctypes.c_int32), ("tile_m", ctypes.c_int32),
                 ("tile_n", ctypes.c_int32), ("num_tiles", ctypes.c_int32),
-                ("grid", ctypes.c_int32), ("waves_x100", ctypes.c_int32)]
+                ("grid", ctypes.c_int32), ("waves_x100", ctypes.c_int32),
+                ("split_tiles", ctypes.c_int32), ("split_kblocks_per_pair", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -64,11 +65,12 @@ _SIGNATURES = {
     "w8a8_version": ([], ctypes.c_char_p),
     "w8a8_quantize_weights": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp], _int),
     "w8a8_quant_act": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp], _int),
+    "w8a8_unpack_int32_weights": ([_vp, _i64, _i64, _vp, _vp], _int),
     "w8a8_workspace_size": ([_i64, _i64, _i64, ctypes.POINTER(_sz)], _int),
     "w8a8_linear": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp],
                     _int),
-    "w8a8_linear_ex": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _int, _vp],
-                       _int),
+    "w8a8_linear_ex": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _int, _vp,
+                        _sz, _vp], _int),
     "w8a8_linear_fused": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp,
                            _vp, _sz, _vp], _int),
     "w8a8_linear_fused_host": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz,
@@ -125,6 +127,10 @@ def w8a8_quantize_weights(W, N, K, ldw, Wq, s_w, stream) -> int:
     return lib().w8a8_quantize_weights(W, N, K, ldw, Wq, s_w, stream)
 
 
+def w8a8_unpack_int32_weights(packed, N, K, Wq, stream) -> int:
+    return lib().w8a8_unpack_int32_weights(packed, N, K, Wq, stream)
+
+
 def w8a8_quant_act(x, M, K, ldx, q, s_a, stream) -> int:
     return lib().w8a8_quant_act(x, M, K, ldx, q, s_a, stream)
 
@@ -141,9 +147,10 @@ def w8a8_linear(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, workspace, ws
                              ws_bytes, stream)
 
 
-def w8a8_linear_ex(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant, stream) -> int:
+def w8a8_linear_ex(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant, workspace,
+                   ws_bytes, stream) -> int:
     return lib().w8a8_linear_ex(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant,
-                                stream)
+                                workspace, ws_bytes, stream)
 
 
 def w8a8_linear_fused(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, q_out, s_a_out, workspace,
@@ -228,6 +235,19 @@ def quantize_weights(W: torch.Tensor, stream=None):
     return Wq, s_w
 
 
+def unpack_int32_weights(packed: torch.Tensor, stream=None) -> torch.Tensor:
+    """Packed int32 [N, K/4] weight storage (codes + 128, four per word, first
+    code in the low byte) -> Wq int8 [N, K] on packed's device."""
+    _need(packed, "packed", torch.int32, 2)
+    if not packed.is_contiguous():
+        raise ValueError("packed must be dense row-major")
+    N, K = packed.shape[0], packed.shape[1] * 4
+    Wq = torch.empty((N, K), dtype=torch.int8, device=packed.device)
+    _check(w8a8_unpack_int32_weights(_ptr(packed), N, K, _ptr(Wq), _stream(stream)),
+           "w8a8_unpack_int32_weights")
+    return Wq
+
+
 def quant_act(x: torch.Tensor, stream=None):
     """bf16 x [M, K] -> (q int8 [M, K], s_a fp32 [M])."""
     _need(x, "x", torch.bfloat16, 2)
@@ -239,10 +259,25 @@ def quant_act(x: torch.Tensor, stream=None):
     return q, s_a
 
 
+def _workspace_for(M, N, K, workspace, dev):
+    """(tensor, pointer, bytes): the caller's workspace, or a fresh one of
+    workspace_size(M, N, K) bytes when `workspace` is None.  The caller keeps
+    the returned tensor alive until the launch has been enqueued: the device
+    memory must not return to the allocator before then, or an output
+    allocated afterwards could share it."""
+    need = workspace_size(M, N, K)
+    if workspace is None:
+        if need == 0:
+            return None, None, 0
+        workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
+    return workspace, _ptr(workspace), workspace.numel() * workspace.element_size()
+
+
 def linear(q, s_a, Wq, s_w, bias=None, out=None, acc_debug=False, variant=VARIANT_AUTO,
-           stream=None):
+           workspace=None, split=True, stream=None):
     """y = bf16(((float)(q @ Wq^T) * s_a) * s_w + bias); with acc_debug=True the raw
-    int32 accumulators [M, N] are returned instead."""
+    int32 accumulators [M, N] are returned instead.  split=False runs the pair
+    kernel without its K-split tail (no workspace is passed)."""
     _need(q, "q", torch.int8, 2)
     dev = q.device
     _need(s_a, "s_a", torch.float32, 1, dev)
@@ -258,15 +293,21 @@ def linear(q, s_a, Wq, s_w, bias=None, out=None, acc_debug=False, variant=VARIAN
         _need(bias, "bias", torch.bfloat16, 1, dev)
         if bias.shape[0] != N:
             raise ValueError("bias must have N elements")
+    ws, ws_ptr, ws_bytes = (_workspace_for(M, N, K, workspace, dev) if split
+                            else (None, None, 0))
     if acc_debug:
         acc = torch.empty((M, N), dtype=torch.int32, device=dev)
         _check(w8a8_linear_ex(_ptr(q), _ptr(s_a), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
-                              None, N, _ptr(acc), variant, _stream(stream)), "w8a8_linear_ex")
+                              None, N, _ptr(acc), variant, ws_ptr, ws_bytes, _stream(stream)),
+               "w8a8_linear_ex")
+        del ws  # enqueued: later allocations on this stream are ordered after the launch
         return acc
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     _need(y, "out", torch.bfloat16, 2, dev)
     _check(w8a8_linear_ex(_ptr(q), _ptr(s_a), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
-                          _ptr(y), y.stride(0), None, variant, _stream(stream)), "w8a8_linear_ex")
+                          _ptr(y), y.stride(0), None, variant, ws_ptr, ws_bytes,
+                          _stream(stream)), "w8a8_linear_ex")
+    del ws
     return y
 
 
@@ -290,15 +331,7 @@ def linear_fused(x, Wq, s_w, bias=None, out=None, workspace=None, return_interme
     if return_intermediates:
         q = torch.empty((M, K), dtype=torch.int8, device=dev)
         s_a = torch.empty((M,), dtype=torch.float32, device=dev)
-    ws_ptr, ws_bytes = None, 0
-    if not return_intermediates:
-        need = workspace_size(M, N, K)
-        if need:
-            if workspace is None:
-                workspace = torch.empty((need,), dtype=torch.uint8, device=dev)
-            if workspace.numel() * workspace.element_size() < need:
-                raise ValueError(f"workspace needs {need} bytes")
-            ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    ws, ws_ptr, ws_bytes = _workspace_for(M, N, K, workspace, dev)
     _check(w8a8_linear_fused(_ptr(x), M, K, x.stride(0), _ptr(Wq), _ptr(s_w), _ptr(bias), N,
                              _ptr(y), y.stride(0), _ptr(q), _ptr(s_a), ws_ptr, ws_bytes,
                              _stream(stream)), "w8a8_linear_fused")

@@ -14,6 +14,7 @@
 #include "../../include/w8a8.h"
 #include "w8a8_gemm.cuh"
 #include "w8a8_gemv.cuh"
+#include "w8a8_pack.cuh"
 #include "w8a8_ptx.cuh"
 #include "w8a8_quant.cuh"
 
@@ -25,6 +26,10 @@ constexpr int kGemmStages256 = 4;  // 4 x 48 KB ring for 128x256 tiles
 constexpr int kGemmStages128 = 6;  // 6 x 32 KB ring for 128x128 tiles
 constexpr int kGemmStagesPair = 6; // 6 x 32 KB ring per CTA for 256x256 pair tiles
 constexpr int kGemmGroupM = 8;
+// K-split tail of the pair kernel (in 128-deep k-blocks): shortest piece a
+// pair takes, and the least tail time the split must save per pair.
+constexpr int64_t kSplitMinPiece = 24;
+constexpr int64_t kSplitMinGain = 24;
 constexpr int64_t kQuantMaxV = 12;  // 16-byte vectors per thread in the quant kernel
 constexpr int kGemvMaxSmem = 232448 - 1024;   // q rows of the GEMV (M * K bytes)
 
@@ -137,12 +142,39 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     if (sms < 2) return W8A8_ERR_UNSUPPORTED_SHAPE;
     const int64_t tiles = cdiv(M, 256) * cdiv(N, 256);
     if (tiles > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
-    const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
+    const int64_t kb = cdiv(K, kBK);
+    // Whole tiles in full waves, then -- when it pays -- the last one to two
+    // waves' tiles shared out along K so that every pair gets the same number
+    // of k-blocks (a problem of less than one wave is shared out entirely).
+    // Every shared-out piece costs about two epilogues (its partial sums
+    // written, or read back and added), some 24 k-blocks of MMA time, so
+    // pieces are at least that long and the split must save at least that
+    // much per pair on the tail.
+    int64_t pairs = sms / 2, tile0 = tiles, per = 0;
+    if (tiles % pairs != 0) {
+      const int64_t full = tiles / pairs;
+      const int64_t t0 = full >= 1 ? (full - 1) * pairs : 0;
+      const int64_t units = (tiles - t0) * kb;
+      int64_t pp = cdiv(units, pairs);
+      if (pp < kSplitMinPiece) pp = kSplitMinPiece;
+      const int64_t tail_unsplit = (cdiv(tiles, pairs) - t0 / pairs) * kb;
+      if (tail_unsplit - pp >= kSplitMinGain && units <= INT32_MAX / 2) {
+        tile0 = t0;
+        per = pp;
+      }
+    }
+    if (tile0 == tiles && tiles < pairs) pairs = tiles;
     plan->tile_m = 256;
     plan->tile_n = 256;
     plan->num_tiles = static_cast<int32_t>(tiles);
     plan->grid = static_cast<int32_t>(2 * pairs);
-    plan->waves_x100 = static_cast<int32_t>(100 * tiles / pairs);
+    if (tile0 < tiles) {
+      plan->split_tiles = static_cast<int32_t>(tiles - tile0);
+      plan->split_kblocks_per_pair = static_cast<int32_t>(per);
+      plan->waves_x100 = static_cast<int32_t>(100 * tile0 / pairs + cdiv(100 * per, kb));
+    } else {
+      plan->waves_x100 = static_cast<int32_t>(100 * tiles / pairs);
+    }
     return W8A8_OK;
   }
   if (v != W8A8_VARIANT_GEMM_BN128 && v != W8A8_VARIANT_GEMM_BN256) return W8A8_ERR_INVALID_ARG;
@@ -155,6 +187,49 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
   plan->grid = static_cast<int32_t>(tiles < sms ? tiles : sms);
   plan->waves_x100 = static_cast<int32_t>(100 * tiles / plan->grid);
   return W8A8_OK;
+}
+
+// ---------------------------------------------------------------- workspace
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+size_t fused_workspace_bytes(int64_t M, int64_t K) {
+  return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
+         align256(static_cast<size_t>(M) * sizeof(float));
+}
+
+// The pair kernel's K-split region: arrival counters (16 per shared-out
+// tile, 64-bit), then the partial-sum slots (split_tiles + pairs - 1 of them,
+// 16 slices of 32 x 128 int32 each).  Nothing in it needs initializing.
+size_t split_counter_bytes(const w8a8_plan &plan) {
+  return align256(static_cast<size_t>(plan.split_tiles) * kSlicesPerTile *
+                  sizeof(unsigned long long));
+}
+size_t split_workspace_bytes(const w8a8_plan &plan) {
+  if (plan.variant != W8A8_VARIANT_GEMM_PAIR || plan.split_tiles == 0) return 0;
+  const size_t slots = static_cast<size_t>(plan.split_tiles) + plan.grid / 2 - 1;
+  return split_counter_bytes(plan) + slots * kSlicesPerTile * kSlotInts * sizeof(int32_t);
+}
+
+// The K-split region handed to the pair kernel; counters == nullptr runs it
+// unsplit.
+struct SplitRegion {
+  unsigned long long *counters = nullptr;
+  int32_t *partials = nullptr;
+};
+
+// Launch tags of the K-split arrival counters: distinct for every launch of
+// the process (a captured graph replays its tag; the counters it leaves are
+// reset to 0, which no tag equals).
+std::atomic<unsigned long long> g_split_epoch{1};
+
+SplitRegion split_region(const w8a8_plan &plan, void *base, size_t bytes) {
+  SplitRegion r;
+  const size_t need = split_workspace_bytes(plan);
+  if (need == 0 || base == nullptr || bytes < need || !aligned16(base)) return r;
+  r.counters = static_cast<unsigned long long *>(base);
+  r.partials = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(base) + split_counter_bytes(plan));
+  return r;
 }
 
 // ---------------------------------------------------------------- TMA maps
@@ -268,8 +343,7 @@ int ensure_smem_limit(int bytes) {
 }
 
 int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q, float *s,
-                 int sms, cudaStream_t stream) {
-  (void)sms;
+                 cudaStream_t stream) {
   const uint16_t *xp = static_cast<const uint16_t *>(x);
   if (rows > INT32_MAX / 2) return W8A8_ERR_UNSUPPORTED_SHAPE;
   // G threads per row (32 .. 256), each holding V <= kQuantMaxV vectors of
@@ -344,7 +418,8 @@ int launch_gemm_t(const w8a8_plan &plan, const int8_t *q, const float *s_a, int6
 template <bool RAW>
 int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, int64_t M,
                      int64_t K, const int8_t *wq, const float *s_w, const void *bias, int64_t N,
-                     void *y, int64_t ldy, int32_t *acc, cudaStream_t stream) {
+                     void *y, int64_t ldy, int32_t *acc, const SplitRegion &split,
+                     cudaStream_t stream) {
   using L = PairLayout<kGemmStagesPair>;
   CUtensorMap ma, mb, my;
   int st = encode_i8_map(&ma, q, M, K, kBM);
@@ -372,11 +447,29 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
   p.y = static_cast<uint16_t *>(y);
   p.ldy = ldy;
   p.acc_out = acc;
+  p.sk_tile0 = plan.num_tiles;
+  p.sk_per = 0;
+  p.sk_units = 0;
+  p.split_partials = nullptr;
+  p.split_counters = nullptr;
+  p.split_epoch = 0;
+  int grid = plan.grid;
+  if (plan.split_tiles > 0 && split.counters != nullptr) {
+    p.sk_tile0 = plan.num_tiles - plan.split_tiles;
+    p.sk_per = plan.split_kblocks_per_pair;
+    p.sk_units = plan.split_tiles * p.k_blocks;
+    p.split_partials = split.partials;
+    p.split_counters = split.counters;
+    p.split_epoch = g_split_epoch.fetch_add(1, std::memory_order_relaxed) & kSplitEpochMask;
+    if (p.split_epoch == 0) p.split_epoch = 1;
+  } else if (plan.split_tiles > 0 && plan.num_tiles < plan.grid / 2) {
+    grid = 2 * plan.num_tiles;  // unsplit and under one wave: one pair per tile
+  }
   constexpr auto kernel = gemm_i8_tcgen05_pair_kernel<kGemmStagesPair, RAW>;
   st = ensure_smem_limit<kernel>(L::kSmemBytes);
   if (st != W8A8_OK) return st;
-  return launch_ex(true, kernel, dim3(plan.grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma,
-                   mb, my, p);
+  return launch_ex(true, kernel, dim3(grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma, mb,
+                   my, p);
 }
 
 template <bool FUSED, bool RAW>
@@ -397,13 +490,6 @@ int launch_gemv_m(const w8a8_plan &plan, const GemvParams &p, int max_smem, int 
   if (p.M <= 8) W8A8_GEMV_CASE(8)
   W8A8_GEMV_CASE(16)
 #undef W8A8_GEMV_CASE
-}
-
-size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
-
-size_t fused_workspace_bytes(int64_t M, int64_t K) {
-  return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
-         align256(static_cast<size_t>(M) * sizeof(float));
 }
 
 __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
@@ -439,9 +525,12 @@ __global__ void __launch_bounds__(256) quant_exhaustive_kernel(unsigned long lon
   if (bad) atomicAdd(&counts[1], bad);
 }
 
+// split_ws / split_ws_bytes: room for the pair kernel's K-split region, or
+// nullptr / 0 (the pair kernel then runs unsplit).
 int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
                 const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
-                int32_t *acc, int variant, cudaStream_t stream) {
+                int32_t *acc, int variant, void *split_ws, size_t split_ws_bytes,
+                cudaStream_t stream) {
   if (!q || !s_a || !Wq || !s_w || (!y && !acc)) return W8A8_ERR_INVALID_ARG;
   int st = check_mk(M, K, K);
   if (st != W8A8_OK) return st;
@@ -474,9 +563,11 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
                : launch_gemv_m<false, false>(plan, p, d->max_smem_optin, d->sms, stream);
   }
   if (plan.variant == W8A8_VARIANT_GEMM_PAIR) {
-    return acc ? launch_gemm_pair<true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc, stream)
+    const SplitRegion split = split_region(plan, split_ws, split_ws_bytes);
+    return acc ? launch_gemm_pair<true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc, split,
+                                        stream)
                : launch_gemm_pair<false>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc,
-                                         stream);
+                                         split, stream);
   }
   if (plan.variant == W8A8_VARIANT_GEMM_BN128) {
     return acc ? launch_gemm_t<128, kGemmStages128, true>(plan, q, s_a, M, K, Wq, s_w, bias, N,
@@ -565,7 +656,24 @@ int w8a8_quantize_weights(const void *W, int64_t N, int64_t K, int64_t ldw, int8
   const DeviceInfo *d = nullptr;
   st = query_device(&d);
   if (st != W8A8_OK) return st;
-  return launch_quant(W, N, K, ldw, Wq, s_w, d->sms, reinterpret_cast<cudaStream_t>(stream));
+  return launch_quant(W, N, K, ldw, Wq, s_w, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8a8_unpack_int32_weights(const int32_t *packed, int64_t N, int64_t K, int8_t *Wq,
+                              w8a8_stream_t stream) {
+  if (!packed || !Wq) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(N, K, K);
+  if (st != W8A8_OK) return st;
+  if (!aligned16(packed) || !aligned16(Wq)) return W8A8_ERR_MISALIGNED;
+  const DeviceInfo *d = nullptr;
+  st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  const int64_t n16 = N * K / 16;
+  const int64_t cap = static_cast<int64_t>(d->sms) * 8;
+  const int64_t grid = cdiv(n16, 256) < cap ? cdiv(n16, 256) : cap;
+  return launch(unpack_int32_weights_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0,
+                reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const uint4 *>(packed),
+                reinterpret_cast<uint4 *>(Wq), n16);
 }
 
 int w8a8_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q, float *s_a,
@@ -578,7 +686,7 @@ int w8a8_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q, 
   const DeviceInfo *d = nullptr;
   st = query_device(&d);
   if (st != W8A8_OK) return st;
-  return launch_quant(x, M, K, ldx, q, s_a, d->sms, reinterpret_cast<cudaStream_t>(stream));
+  return launch_quant(x, M, K, ldx, q, s_a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_select(int64_t M, int64_t N, int64_t K, int32_t num_sms, int variant,
@@ -601,26 +709,27 @@ int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes) {
   w8a8_plan plan;
   st = select_plan(M, N, K, 148, W8A8_VARIANT_AUTO, 232448, &plan);
   if (st != W8A8_OK) return st;
-  *bytes = plan.variant == W8A8_VARIANT_GEMV ? 0 : fused_workspace_bytes(M, K);
+  *bytes = plan.variant == W8A8_VARIANT_GEMV
+               ? 0
+               : fused_workspace_bytes(M, K) + split_workspace_bytes(plan);
   return W8A8_OK;
 }
 
 int w8a8_linear(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
                 const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
                 int32_t *acc_debug, void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
-  (void)workspace;
-  (void)ws_bytes;
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, W8A8_VARIANT_AUTO,
-                     reinterpret_cast<cudaStream_t>(stream));
+                     workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
                    const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
-                   int32_t *acc_debug, int variant, w8a8_stream_t stream) {
+                   int32_t *acc_debug, int variant, void *workspace, size_t ws_bytes,
+                   w8a8_stream_t stream) {
   if (variant < W8A8_VARIANT_AUTO || variant > W8A8_VARIANT_GEMM_PAIR)
     return W8A8_ERR_INVALID_ARG;
-  return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant,
-                     reinterpret_cast<cudaStream_t>(stream));
+  return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant, workspace,
+                     ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t *Wq,
@@ -661,18 +770,26 @@ int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const in
     return launch_gemv_m<true, false>(plan, p, d->max_smem_optin, d->sms, stream);
   }
 
+  // workspace layout: [q (M*K) | s_a (M floats) | K-split region]
   int8_t *q = q_out;
   float *s_a = s_a_out;
+  const size_t qs_bytes = fused_workspace_bytes(M, K);
   if (!q || !s_a) {
-    const size_t need = fused_workspace_bytes(M, K);
-    if (!workspace || ws_bytes < need || !aligned16(workspace)) return W8A8_ERR_WORKSPACE;
+    if (!workspace || ws_bytes < qs_bytes || !aligned16(workspace)) return W8A8_ERR_WORKSPACE;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     if (!q) q = reinterpret_cast<int8_t *>(ws);
     if (!s_a) s_a = reinterpret_cast<float *>(ws + align256(static_cast<size_t>(M * K)));
   }
-  st = launch_quant(x, M, K, ldx, q, s_a, d->sms, stream);
+  void *split_ws = nullptr;
+  size_t split_bytes = 0;
+  if (workspace && ws_bytes > qs_bytes && aligned16(workspace)) {
+    split_ws = static_cast<uint8_t *>(workspace) + qs_bytes;
+    split_bytes = ws_bytes - qs_bytes;
+  }
+  st = launch_quant(x, M, K, ldx, q, s_a, stream);
   if (st != W8A8_OK) return st;
-  return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, nullptr, plan.variant, stream);
+  return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, nullptr, plan.variant, split_ws,
+                     split_bytes, stream);
 }
 
 int w8a8_linear_fused_noalloc(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t *Wq,

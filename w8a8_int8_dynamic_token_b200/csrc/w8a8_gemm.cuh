@@ -73,7 +73,95 @@ struct GemmParams {
   uint16_t *y;           // bf16 bits
   int64_t ldy;
   int32_t *acc_out;      // raw int32 [M, N] dense (debug variant)
+  // CTA-pair kernel only.  Tiles [0, sk_tile0) are whole-tile work in full
+  // waves; the remaining tiles (the last one to two waves) are shared out
+  // along K: their k-blocks, in (tile, k-block) order, form sk_units units,
+  // and pair j takes the units [j * sk_per, (j + 1) * sk_per).  A tile worked
+  // on by several pairs is finished by the last of them to arrive (per
+  // epilogue warp slice, elected by an arrival counter), which adds the
+  // others' int32 partial sums from split_partials.
+  int32_t sk_tile0;        // == num_tiles: nothing is split
+  int32_t sk_per;          // units per pair (>= 1)
+  int32_t sk_units;        // (num_tiles - sk_tile0) * k_blocks
+  int32_t *split_partials; // (num_tiles - sk_tile0 + pairs - 1) slots of 16 slices
+  // (num_tiles - sk_tile0) x 16 counters, each (tag << 8) | arrivals.  A
+  // counter whose tag is not this launch's split_epoch counts as 0, so the
+  // memory needs no clearing; the electing contribution resets it to 0.
+  unsigned long long *split_counters;
+  unsigned long long split_epoch;  // 1 .. 2^56 - 1
 };
+
+constexpr unsigned long long kSplitEpochMask = (1ull << 56) - 1;
+
+// One epilogue warp slice of a 256 x 256 pair tile: 32 rows x 128 columns.
+constexpr int kSlotInts = 32 * 128;
+constexpr int kSlicesPerTile = 16;  // 2 CTAs x 8 epilogue warps
+
+// The i-th work item of a CTA pair: a whole tile, or a run of k-blocks of a
+// tile of the shared-out region.  Returns false past the pair's last item.
+struct WorkItem {
+  int tile;        // tile index (row/column block via pair_tile_coords)
+  int kb_begin, kb_end;
+  int t_rel;       // tile - sk_tile0 (shared-out tiles only)
+  int nparts;      // pairs contributing to this tile (1: whole tile)
+  int part;        // this pair's index among them, in k order
+};
+
+__device__ __forceinline__ bool pair_work_item(const GemmParams &p, int pair_id, int num_pairs,
+                                               int i, WorkItem &w) {
+  const int n_dp =
+      pair_id < p.sk_tile0 ? (p.sk_tile0 - pair_id + num_pairs - 1) / num_pairs : 0;
+  if (i < n_dp) {
+    w.tile = pair_id + i * num_pairs;
+    w.kb_begin = 0;
+    w.kb_end = p.k_blocks;
+    w.t_rel = -1;
+    w.nparts = 1;
+    w.part = 0;
+    return true;
+  }
+  if (p.sk_tile0 >= p.num_tiles) return false;
+  const int kb = p.k_blocks;
+  const int u0 = pair_id * p.sk_per;
+  const int u1 = min(u0 + p.sk_per, p.sk_units);
+  if (u0 >= u1) return false;
+  const int t_rel = u0 / kb + (i - n_dp);
+  if (t_rel * kb >= u1) return false;
+  w.t_rel = t_rel;
+  w.tile = p.sk_tile0 + t_rel;
+  w.kb_begin = max(u0 - t_rel * kb, 0);
+  w.kb_end = min(u1 - t_rel * kb, kb);
+  const int first = (t_rel * kb) / p.sk_per;
+  const int last = ((t_rel + 1) * kb - 1) / p.sk_per;
+  w.nparts = last - first + 1;
+  w.part = pair_id - first;
+  return true;
+}
+
+// Registers one arrival on a K-split counter for launch tag `epoch`; returns
+// how many contributions had arrived before (-1 if the retry bound ran out,
+// which also sets the device error word).
+__device__ __forceinline__ int split_arrive(unsigned long long *counter, unsigned long long epoch) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(counter);
+  for (int i = 0; i < (1 << 20); ++i) {
+    const unsigned long long before = (cur >> 8) == epoch ? (cur & 0xFFull) : 0ull;
+    const unsigned long long prev = atomicCAS(counter, cur, (epoch << 8) | (before + 1ull));
+    if (prev == cur) return static_cast<int>(before);
+    cur = prev;
+  }
+  atomicOr(&g_device_error, W8A8_DEVERR_TIMEOUT);
+  return -1;
+}
+
+// Partial-sum slice of pair `pair` on shared-out tile t_rel.  Slot t_rel +
+// pair is unique: two contributions (t, j) and (t + d, j - d), d >= 1, cannot
+// both exist, since pair j - d ends at or before unit j * sk_per, which is
+// below (t + 1) * k_blocks, where tile t + d starts at the earliest.
+__device__ __forceinline__ int32_t *split_slice(const GemmParams &p, int t_rel, int pair,
+                                                int slice) {
+  return p.split_partials +
+         (static_cast<int64_t>(t_rel + pair) * kSlicesPerTile + slice) * kSlotInts;
+}
 
 // Tile t -> (row block, column block).  Row blocks are walked in bands of
 // group_m so the tiles in flight at one time share their q and Wq slices in L2.
@@ -97,11 +185,20 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) 
 // One epilogue warp's share of an accumulator: its 32 TMEM lanes (tile rows
 // row0 .. row0+31) and COLS columns starting at output column col_base, in
 // chunks of 32 columns.  t_row addresses (first lane, first column).
+// Modes: kEpiNormal -- the epilogue proper; kEpiWritePartial -- store the
+// raw int32 accumulators to the slice at `slot` and nothing else;
+// kEpiAddPartials -- add the slices at slot + j * part_stride, j < nparts,
+// j != own_part, to the accumulators (exact int32 sums), then the epilogue
+// proper.
+constexpr int kEpiNormal = 0, kEpiWritePartial = 1, kEpiAddPartials = 2;
+
 template <int COLS, bool RAW_OUT>
 __device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const CUtensorMap *tmap_y,
                                                     uint32_t t_row, int row0, int col_base,
                                                     uint8_t *stage_buf, uint32_t &chunk_count,
-                                                    int lane) {
+                                                    int lane, int mode = kEpiNormal,
+                                                    int32_t *slot = nullptr, int nparts = 0,
+                                                    int own_part = 0, int64_t part_stride = 0) {
   const int row = row0 + lane;
   const bool row_ok = row < p.M;
   const float sa = row_ok ? __ldg(p.s_a + row) : 0.0f;
@@ -111,10 +208,33 @@ __device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const C
   for (int c = 0; c < cols_here; c += kEpiChunk) {
     const int col0 = col_base + c;
     if (col0 >= p.N) break;  // warp-uniform
+    if (mode == kEpiWritePartial) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(t_row + c, r);
+      tmem_ld_wait();
+      // slice layout: uint4 index ((c / 32) * 8 + g) * 32 + lane (coalesced)
+      uint4 *dst = reinterpret_cast<uint4 *>(slot) + (c / 32) * 256 + lane;
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        __stcg(dst + 32 * g, make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]));
+      continue;
+    }
     if constexpr (RAW_OUT) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(t_row + c, r);
       tmem_ld_wait();
+      if (mode == kEpiAddPartials) {
+        for (int j = 0; j < nparts; ++j) {
+          if (j == own_part) continue;
+          const uint4 *src =
+              reinterpret_cast<const uint4 *>(slot + j * part_stride) + (c / 32) * 256 + lane;
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const uint4 a = __ldcg(src + 32 * g);
+            r[4 * g] += a.x; r[4 * g + 1] += a.y; r[4 * g + 2] += a.z; r[4 * g + 3] += a.w;
+          }
+        }
+      }
       if (row_ok) {
         int32_t *dst = p.acc_out + static_cast<int64_t>(row) * p.N + col0;
 #pragma unroll
@@ -154,6 +274,18 @@ __device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const C
       uint32_t r[32];
       tmem_ld_32x32b_x32(t_row + c, r);
       tmem_ld_wait();
+      if (mode == kEpiAddPartials) {  // exact int32 sum of the K-parts
+        for (int j = 0; j < nparts; ++j) {
+          if (j == own_part) continue;
+          const uint4 *src =
+              reinterpret_cast<const uint4 *>(slot + j * part_stride) + (c / 32) * 256 + lane;
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const uint4 a = __ldcg(src + 32 * g);
+            r[4 * g] += a.x; r[4 * g + 1] += a.y; r[4 * g + 2] += a.z; r[4 * g + 3] += a.w;
+          }
+        }
+      }
       // two adjacent columns at a time in packed fp32: each lane of every
       // packed operation is the same separately rounded operation as before
       uint32_t packed[16];
@@ -481,22 +613,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // Wq loads of the first ring's worth of stages before waiting for the
       // preceding kernel (programmatic dependent launch); q after the wait.
       int prefetched = 0;
-      if (pair_id < p.num_tiles) {
+      WorkItem w;
+      if (pair_work_item(p, pair_id, num_pairs, 0, w)) {
         int mb0, nb0;
-        pair_tile_coords(pair_id, p, mb0, nb0);
-        prefetched = p.k_blocks < STAGES ? p.k_blocks : STAGES;
-        for (int kb = 0; kb < prefetched; ++kb) {
-          uint8_t *sb = smem + kb * L::kStageBytes + L::kABytes;
-          if (rank == 0) mbar_arrive_expect_tx(&full[kb], 2 * L::kStageBytes);
-          tma_load_2d_pair(&tmap_b, map_to_cta(smem_addr(&full[kb]), 0), sb, kb * kBK,
-                           nb0 * kPairBN + static_cast<int>(rank) * 128);
+        pair_tile_coords(w.tile, p, mb0, nb0);
+        const int nkb = w.kb_end - w.kb_begin;
+        prefetched = nkb < STAGES ? nkb : STAGES;
+        for (int i = 0; i < prefetched; ++i) {
+          uint8_t *sb = smem + i * L::kStageBytes + L::kABytes;
+          if (rank == 0) mbar_arrive_expect_tx(&full[i], 2 * L::kStageBytes);
+          tma_load_2d_pair(&tmap_b, map_to_cta(smem_addr(&full[i]), 0), sb,
+                           (w.kb_begin + i) * kBK, nb0 * kPairBN + static_cast<int>(rank) * 128);
         }
       }
       grid_dependency_wait();
-      for (int t = pair_id; ok && t < p.num_tiles; t += num_pairs) {
+      for (int it = 0; ok && pair_work_item(p, pair_id, num_pairs, it, w); ++it) {
         int mb, nb;
-        pair_tile_coords(t, p, mb, nb);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        pair_tile_coords(w.tile, p, mb, nb);
+        for (int kb = w.kb_begin; kb < w.kb_end; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -536,14 +670,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       bool any_mma = false;
-      for (int t = pair_id; ok && t < p.num_tiles; t += num_pairs) {
+      WorkItem w;
+      for (int it = 0; ok && pair_work_item(p, pair_id, num_pairs, it, w); ++it) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPairBN);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = w.kb_begin; kb < w.kb_end; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             ok = false;
             break;
@@ -554,7 +689,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint64_t bdesc = smem_desc_k_sw128(sa + L::kABytes);
 #pragma unroll
           for (int k = 0; k < kBK / kMmaK; ++k)
-            mma_i8_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            mma_i8_pair(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc,
+                        (kb != w.kb_begin || k != 0) ? 1u : 0u);
           any_mma = true;
           mma_commit_pair(&empty[stage], 0x3);
           if (++stage == STAGES) {
@@ -583,10 +719,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t chunk_count = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
+    const int slice = static_cast<int>(rank) * kEpiWarps + e;
     grid_dependency_wait();  // s_a comes from the preceding kernel
-    for (int t = pair_id; t < p.num_tiles; t += num_pairs) {
+    WorkItem w;
+    for (int it = 0; pair_work_item(p, pair_id, num_pairs, it, w); ++it) {
       int mb, nb;
-      pair_tile_coords(t, p, mb, nb);
+      pair_tile_coords(w.tile, p, mb, nb);
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], acc_phase, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -594,9 +732,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * kPairBN + half * (kPairBN / 2));
-      epilogue_warp_slice<kPairBN / 2, RAW_OUT>(
-          p, &tmap_y, t_row, mb * 256 + static_cast<int>(rank) * 128 + quarter * 32,
-          nb * kPairBN + half * (kPairBN / 2), stage_buf, chunk_count, lane);
+      const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
+      const int col_base = nb * kPairBN + half * (kPairBN / 2);
+      if (w.nparts == 1) {
+        epilogue_warp_slice<kPairBN / 2, RAW_OUT>(p, &tmap_y, t_row, row0, col_base, stage_buf,
+                                                  chunk_count, lane);
+      } else {
+        // Shared-out tile: the last contribution to arrive finishes it.  The
+        // part holding k-block 0 is this pair's last item and usually the
+        // last to arrive: if all the others are in already it skips writing
+        // its own partial sums.
+        unsigned long long *counter = p.split_counters + w.t_rel * kSlicesPerTile + slice;
+        int32_t *first_slice = split_slice(p, w.t_rel, pair_id - w.part, slice);
+        const unsigned long long all_others =
+            (p.split_epoch << 8) | static_cast<unsigned long long>(w.nparts - 1);
+        int last = 0;
+        if (w.part == 0 && lane == 0) last = ld_acquire_gpu_u64(counter) == all_others ? 1 : 0;
+        __syncwarp();  // orders the lanes' partial-sum reads after lane 0's acquire
+        last = __shfl_sync(0xFFFFFFFFu, last, 0);
+        if (!last) {
+          epilogue_warp_slice<kPairBN / 2, RAW_OUT>(
+              p, &tmap_y, t_row, row0, col_base, stage_buf, chunk_count, lane, kEpiWritePartial,
+              first_slice + static_cast<int64_t>(w.part) * kSlicesPerTile * kSlotInts);
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) last = split_arrive(counter, p.split_epoch) == w.nparts - 1 ? 1 : 0;
+          __syncwarp();
+          last = __shfl_sync(0xFFFFFFFFu, last, 0);
+        }
+        if (last) {
+          __threadfence();
+          if (lane == 0) *reinterpret_cast<volatile unsigned long long *>(counter) = 0ull;
+          epilogue_warp_slice<kPairBN / 2, RAW_OUT>(
+              p, &tmap_y, t_row, row0, col_base, stage_buf, chunk_count, lane, kEpiAddPartials,
+              first_slice, w.nparts, w.part, static_cast<int64_t>(kSlicesPerTile) * kSlotInts);
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_cta(smem_addr(&tempty[acc]), 0));
