@@ -310,7 +310,8 @@ def cpu_baseline(case: synth.LayerCase, budget_s: float = 12.0, max_rows: int = 
     x = case.x()
     wq, sw = oracle.quantize_weights(case.w())
     b = case.b()
-    rows = 4
+    # calibrate on one row per oracle thread (it parallelizes over rows)
+    rows = int(max(4, min(M, oracle.threads())))
     t0 = time.perf_counter()
     oracle.linear(x[:rows], wq, sw, b)
     dt = time.perf_counter() - t0
