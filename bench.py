@@ -91,7 +91,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.ok = False
         self.samples, self.reasons = [], 0
         self.period = period_s
@@ -118,6 +118,10 @@ class ClockSampler:
 
     def __enter__(self):
         if self.ok:
+            # the launching thread holds the GIL most of the time: hand it
+            # over more often so the sampler runs at its period
+            self._switch = sys.getswitchinterval()
+            sys.setswitchinterval(2e-4)
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
@@ -126,6 +130,7 @@ class ClockSampler:
         if self.ok:
             self._stop.set()
             self.t.join()
+            sys.setswitchinterval(self._switch)
 
     def summary(self):
         if not self.ok:
