@@ -99,6 +99,9 @@ typedef struct {
                               0 = none */
     int32_t split_kblocks_per_pair; /* GEMM_PAIR with split_tiles > 0: 128-deep
                               k-blocks of that region per pair, else 0 */
+    int32_t tail_tiles_nsplit; /* GEMM_PAIR: 2 when the tiles of the last,
+                              partial round are cut along N into two
+                              128-column tiles (one per pair); else 0 */
 } w8a8_plan;
 
 /* Human-readable name of a status code (static string, never NULL). */

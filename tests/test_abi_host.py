@@ -135,9 +135,16 @@ def test_workspace_size_covers_q_and_scales():
 # model of the device-side partition (work items, contributor counts, partial
 # slots) checks that every (tile, k-block) is computed exactly once and that
 # the partial-sum slots of different contributions never collide.
-def _pair_items(tiles, split_tiles, per, kb, pairs, pair):
+def _pair_items(tiles, split_tiles, per, kb, pairs, pair, nsplit=0):
+    if nsplit > 1:   # whole tiles in full rounds, then one narrow tail tile per pair
+        tile0 = tiles - tiles % pairs
+        items = [(t, 0, kb, 1, 0, 0, 256) for t in range(pair, tile0, pairs)]
+        if pair < (tiles - tile0) * nsplit:
+            w = 256 // nsplit
+            items.append((tile0 + pair // nsplit, 0, kb, 1, 0, (pair % nsplit) * w, w))
+        return items
     tile0 = tiles - split_tiles
-    items = [(t, 0, kb, 1, 0) for t in range(pair, tile0, pairs)]
+    items = [(t, 0, kb, 1, 0, 0, 256) for t in range(pair, tile0, pairs)]
     if split_tiles:
         units = split_tiles * kb
         u0, u1 = pair * per, min(pair * per + per, units)
@@ -145,7 +152,7 @@ def _pair_items(tiles, split_tiles, per, kb, pairs, pair):
         while t is not None and t * kb < u1:
             first, last = (t * kb) // per, ((t + 1) * kb - 1) // per
             items.append((tile0 + t, max(u0 - t * kb, 0), min(u1 - t * kb, kb),
-                          last - first + 1, pair - first))
+                          last - first + 1, pair - first, 0, 256))
             t += 1
     return items
 
@@ -166,23 +173,41 @@ def test_pair_k_split_partition(M, N, K):
     if st:
         assert per >= 24 and per * pairs >= st * kb
         assert st <= tiles and (tiles - st) % pairs == 0 and st < 2 * pairs
+    ns = p["tail_tiles_nsplit"]
+    assert not (ns and st)
     covered = {}
     slots = set()
     for pair in range(pairs):
-        for t, b, e, nparts, part in _pair_items(tiles, st, per, kb, pairs, pair):
+        for t, b, e, nparts, part, n0, w in _pair_items(tiles, st, per, kb, pairs, pair, ns):
             assert 0 <= b < e <= kb and 0 <= part < nparts
             for k in range(b, e):
-                assert (t, k) not in covered
-                covered[(t, k)] = pair
+                for c in range(n0 // 64, (n0 + w) // 64):   # 64-column granules
+                    assert (t, k, c) not in covered
+                    covered[(t, k, c)] = pair
+                covered.setdefault((t, k), pair)
             if nparts > 1:
                 slot = (t - (tiles - st)) + pair
                 assert slot not in slots and slot < st + pairs - 1
                 slots.add(slot)
-    assert len(covered) == tiles * kb
+    assert sum(1 for key in covered if len(key) == 3) == tiles * kb * 4
     # contributor counts agree with who actually covers each tile
     for t in range(tiles - st, tiles):
         owners = sorted({covered[(t, k)] for k in range(kb)})
         assert owners == list(range(owners[0], owners[-1] + 1))
+
+
+def test_pair_n_split_tail_plans():
+    # QKV: 612 tiles = 8 rounds of 74 + 20; the 20 are cut in halves (40 <= 74)
+    p = w8a8.select(4352, 9216, 3072)
+    assert p["tail_tiles_nsplit"] == 2 and p["split_tiles"] == 0 and p["waves_x100"] == 850
+    # FFN up: 816 = 11 x 74 + 2 -> halves
+    p = w8a8.select(4352, 12288, 3072)
+    assert p["tail_tiles_nsplit"] == 2 and p["waves_x100"] == 1150
+    # a last round more than half full cannot be shortened by cutting along N
+    assert w8a8.select(4352, 3072, 12288)["tail_tiles_nsplit"] == 0    # 204 = 2 x 74 + 56
+    assert w8a8.select(8704, 3072, 12288)["tail_tiles_nsplit"] == 0    # 408 = 5 x 74 + 38
+    # under one round there is no tail to cut
+    assert w8a8.select(512, 9216, 3072, variant=B.VARIANT_GEMM_PAIR)["tail_tiles_nsplit"] == 0
 
 
 def test_pair_k_split_plans():
@@ -192,7 +217,7 @@ def test_pair_k_split_plans():
     assert p["variant_name"] == "gemm_pair"
     assert p["split_tiles"] == 408 - 4 * 74 and p["split_kblocks_per_pair"] == -(-112 * 96 // 74)
     assert p["waves_x100"] == 400 + -(-100 * 146 // 96)
-    # short tiles: shared-out pieces would be epilogue-bound -> no split
+    # short tiles: shared-out pieces would be epilogue-bound -> no K split
     for M, N, K in ((4352, 9216, 3072), (4352, 12288, 3072), (8704, 3072, 3072)):
         assert w8a8.select(M, N, K)["split_tiles"] == 0
     # a tail that is already three quarters full: the split saves too little

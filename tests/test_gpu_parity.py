@@ -522,3 +522,32 @@ def test_dit_block_linears_back_to_back():
         rows = sample_rows(c.M, seed=c.seed, n_random=32, tile=256)
         r = oracle.linear(np.ascontiguousarray(x[rows]), wq, sw, b)
         assert check_y(bits_of(y)[rows], r["y"], r["y32"], c.name) == 0
+
+
+# ----------------------------------------------------------------- N-split tail
+
+# (M, N, K): 76 tiles = one round + 2, ragged M and a ragged last column
+# block (500 x 9720); 94 tiles = one round + 20 (512 x 12032).
+NSPLIT_CASES = [(500, 9720, 512, 2), (512, 12032, 512, 2)]
+
+
+@pytest.mark.parametrize("M,N,K,nsplit", NSPLIT_CASES)
+def test_pair_n_split_tail_exact(M, N, K, nsplit):
+    """The pair kernel with the tiles of its last round cut along N into
+    narrower tiles: raw int32 accumulators and y against the oracle, in full."""
+    assert w8a8.select(M, N, K, variant=B.VARIANT_GEMM_PAIR)["tail_tiles_nsplit"] == nsplit
+    rng = np.random.default_rng(M * 3 + N + K)
+    q = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
+    wq = rng.integers(-127, 128, size=(N, K), dtype=np.int8)
+    s_a = (rng.random(M, dtype=np.float32) * 0.05 + 1e-3).astype(np.float32)
+    s_w = (rng.random(N, dtype=np.float32) * 0.002 + 1e-4).astype(np.float32)
+    b = synth.make_bias(N, seed=6)
+    args = (torch.from_numpy(q).cuda(), torch.from_numpy(s_a).cuda(), torch.from_numpy(wq).cuda(),
+            torch.from_numpy(s_w).cuda(), to_dev(b))
+    acc = w8a8.linear(*args, acc_debug=True, variant=B.VARIANT_GEMM_PAIR)
+    y = w8a8.linear(*args, variant=B.VARIANT_GEMM_PAIR)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_i32(q, wq)
+    assert np.array_equal(acc.cpu().numpy(), ref)
+    y32, y_ref = oracle.epilogue(ref, s_a, s_w, b)
+    assert check_y(bits_of(y), y_ref, y32, "n-split") == 0

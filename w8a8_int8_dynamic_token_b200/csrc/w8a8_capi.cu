@@ -150,9 +150,16 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     // written, or read back and added), some 24 k-blocks of MMA time, so
     // pieces are at least that long and the split must save at least that
     // much per pair on the tail.
-    int64_t pairs = sms / 2, tile0 = tiles, per = 0;
-    if (tiles % pairs != 0) {
-      const int64_t full = tiles / pairs;
+    int64_t pairs = sms / 2, tile0 = tiles, per = 0, nsplit = 1;
+    const int64_t full = tiles / pairs, rem = tiles % pairs;
+    if (full >= 1 && rem > 0 && 2 * rem <= pairs) {
+      // A last round of rem tiles on `pairs` pairs costs as much as a full
+      // round: cut each of its tiles along N into two 128-column tiles, one
+      // per pair.  (Narrow tiles read more operand bytes per MMA; at 64
+      // columns the round becomes bandwidth-bound and gains nothing.)
+      nsplit = 2;
+      tile0 = full * pairs;
+    } else if (rem != 0) {
       const int64_t t0 = full >= 1 ? (full - 1) * pairs : 0;
       const int64_t units = (tiles - t0) * kb;
       int64_t pp = cdiv(units, pairs);
@@ -168,7 +175,10 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     plan->tile_n = 256;
     plan->num_tiles = static_cast<int32_t>(tiles);
     plan->grid = static_cast<int32_t>(2 * pairs);
-    if (tile0 < tiles) {
+    if (nsplit > 1) {
+      plan->tail_tiles_nsplit = static_cast<int32_t>(nsplit);
+      plan->waves_x100 = static_cast<int32_t>(100 * full + 100 / nsplit);
+    } else if (tile0 < tiles) {
       plan->split_tiles = static_cast<int32_t>(tiles - tile0);
       plan->split_kblocks_per_pair = static_cast<int32_t>(per);
       plan->waves_x100 = static_cast<int32_t>(100 * tile0 / pairs + cdiv(100 * per, kb));
@@ -421,11 +431,19 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
                      void *y, int64_t ldy, int32_t *acc, const SplitRegion &split,
                      cudaStream_t stream) {
   using L = PairLayout<kGemmStagesPair>;
-  CUtensorMap ma, mb, my;
+  CUtensorMap ma, mb, mbt, my;
   int st = encode_i8_map(&ma, q, M, K, kBM);
   if (st != W8A8_OK) return st;
   st = encode_i8_map(&mb, wq, N, K, kPairBN / 2);
   if (st != W8A8_OK) return st;
+  // narrow tail tiles: each CTA loads (256 / nsplit) / 2 rows of Wq per stage
+  const int nsplit = plan.tail_tiles_nsplit > 1 ? plan.tail_tiles_nsplit : 1;
+  if (nsplit > 1) {
+    st = encode_i8_map(&mbt, wq, N, K, kPairBN / 2 / nsplit);
+    if (st != W8A8_OK) return st;
+  } else {
+    mbt = mb;
+  }
   if (RAW) {
     std::memset(&my, 0, sizeof(my));
   } else {
@@ -447,15 +465,19 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
   p.y = static_cast<uint16_t *>(y);
   p.ldy = ldy;
   p.acc_out = acc;
-  p.sk_tile0 = plan.num_tiles;
+  p.dp_tiles = plan.num_tiles;
+  p.tail_nsplit = 1;
   p.sk_per = 0;
   p.sk_units = 0;
   p.split_partials = nullptr;
   p.split_counters = nullptr;
   p.split_epoch = 0;
   int grid = plan.grid;
-  if (plan.split_tiles > 0 && split.counters != nullptr) {
-    p.sk_tile0 = plan.num_tiles - plan.split_tiles;
+  if (nsplit > 1) {
+    p.tail_nsplit = nsplit;
+    p.dp_tiles = plan.num_tiles - plan.num_tiles % (plan.grid / 2);
+  } else if (plan.split_tiles > 0 && split.counters != nullptr) {
+    p.dp_tiles = plan.num_tiles - plan.split_tiles;
     p.sk_per = plan.split_kblocks_per_pair;
     p.sk_units = plan.split_tiles * p.k_blocks;
     p.split_partials = split.partials;
@@ -469,7 +491,7 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
   st = ensure_smem_limit<kernel>(L::kSmemBytes);
   if (st != W8A8_OK) return st;
   return launch_ex(true, kernel, dim3(grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma, mb,
-                   my, p);
+                   mbt, my, p);
 }
 
 template <bool FUSED, bool RAW>

@@ -47,6 +47,7 @@ constexpr int kEpiBufBytes = 32 * kEpiChunk * 2;  // 32 rows x 32 bf16
 constexpr int kBM = 128;   // rows of y per tile (TMEM lanes)
 constexpr int kBK = 128;   // int8 K elements per stage = one 128-byte swizzle row
 constexpr int kMmaK = 32;  // K per tcgen05.mma kind::i8
+constexpr int kPairBN = 256;  // columns of a CTA-pair tile
 
 template <int BN, int STAGES>
 struct GemmLayout {
@@ -73,18 +74,23 @@ struct GemmParams {
   uint16_t *y;           // bf16 bits
   int64_t ldy;
   int32_t *acc_out;      // raw int32 [M, N] dense (debug variant)
-  // CTA-pair kernel only.  Tiles [0, sk_tile0) are whole-tile work in full
-  // waves; the remaining tiles (the last one to two waves) are shared out
-  // along K: their k-blocks, in (tile, k-block) order, form sk_units units,
-  // and pair j takes the units [j * sk_per, (j + 1) * sk_per).  A tile worked
-  // on by several pairs is finished by the last of them to arrive (per
-  // epilogue warp slice, elected by an arrival counter), which adds the
-  // others' int32 partial sums from split_partials.
-  int32_t sk_tile0;        // == num_tiles: nothing is split
-  int32_t sk_per;          // units per pair (>= 1)
-  int32_t sk_units;        // (num_tiles - sk_tile0) * k_blocks
-  int32_t *split_partials; // (num_tiles - sk_tile0 + pairs - 1) slots of 16 slices
-  // (num_tiles - sk_tile0) x 16 counters, each (tag << 8) | arrivals.  A
+  // CTA-pair kernel only.  Tiles [0, dp_tiles) are whole-tile work in full
+  // rounds (pair j takes tiles j, j + pairs, ...).  The remaining tiles, when
+  // there are any, form the tail, handled in one of two ways:
+  //  - split along N (tail_nsplit = 2 or 4): each tail tile becomes
+  //    tail_nsplit tiles 256/tail_nsplit columns wide, one per pair;
+  //  - split along K (sk_per > 0): their k-blocks, in (tile, k-block) order,
+  //    form sk_units units and pair j takes the units [j * sk_per,
+  //    (j + 1) * sk_per).  A tile worked on by several pairs is finished by
+  //    the last of them to arrive (per epilogue warp slice, elected by an
+  //    arrival counter), which adds the others' int32 partial sums from
+  //    split_partials.
+  int32_t dp_tiles;        // == num_tiles: no tail
+  int32_t tail_nsplit;     // 1 (no N split), 2 or 4
+  int32_t sk_per;          // K split: units per pair, 0 = no K split
+  int32_t sk_units;        // (num_tiles - dp_tiles) * k_blocks
+  int32_t *split_partials; // (num_tiles - dp_tiles + pairs - 1) slots of 16 slices
+  // (num_tiles - dp_tiles) x 16 counters, each (tag << 8) | arrivals.  A
   // counter whose tag is not this launch's split_epoch counts as 0, so the
   // memory needs no clearing; the electing contribution resets it to 0.
   unsigned long long *split_counters;
@@ -97,30 +103,45 @@ constexpr unsigned long long kSplitEpochMask = (1ull << 56) - 1;
 constexpr int kSlotInts = 32 * 128;
 constexpr int kSlicesPerTile = 16;  // 2 CTAs x 8 epilogue warps
 
-// The i-th work item of a CTA pair: a whole tile, or a run of k-blocks of a
-// tile of the shared-out region.  Returns false past the pair's last item.
+// The i-th work item of a CTA pair: a whole tile, a narrow tail tile (a
+// column range of a tile), or a run of k-blocks of a tile shared out along K.
+// Returns false past the pair's last item.
 struct WorkItem {
   int tile;        // tile index (row/column block via pair_tile_coords)
   int kb_begin, kb_end;
-  int t_rel;       // tile - sk_tile0 (shared-out tiles only)
-  int nparts;      // pairs contributing to this tile (1: whole tile)
+  int n_off;       // first column of the item within the tile
+  int ncols;       // columns of the item: 256, or 256 / tail_nsplit
+  int t_rel;       // tile - dp_tiles (K-split tiles only)
+  int nparts;      // pairs contributing to this tile along K (1: all of K)
   int part;        // this pair's index among them, in k order
 };
 
 __device__ __forceinline__ bool pair_work_item(const GemmParams &p, int pair_id, int num_pairs,
                                                int i, WorkItem &w) {
   const int n_dp =
-      pair_id < p.sk_tile0 ? (p.sk_tile0 - pair_id + num_pairs - 1) / num_pairs : 0;
+      pair_id < p.dp_tiles ? (p.dp_tiles - pair_id + num_pairs - 1) / num_pairs : 0;
+  w.n_off = 0;
+  w.ncols = kPairBN;
+  w.t_rel = -1;
+  w.nparts = 1;
+  w.part = 0;
   if (i < n_dp) {
     w.tile = pair_id + i * num_pairs;
     w.kb_begin = 0;
     w.kb_end = p.k_blocks;
-    w.t_rel = -1;
-    w.nparts = 1;
-    w.part = 0;
     return true;
   }
-  if (p.sk_tile0 >= p.num_tiles) return false;
+  if (p.dp_tiles >= p.num_tiles) return false;
+  if (p.tail_nsplit > 1) {  // one narrow tail tile per pair, pairs 0 .. R * nsplit - 1
+    if (i != n_dp || pair_id >= (p.num_tiles - p.dp_tiles) * p.tail_nsplit) return false;
+    w.tile = p.dp_tiles + pair_id / p.tail_nsplit;
+    w.ncols = kPairBN / p.tail_nsplit;
+    w.n_off = (pair_id % p.tail_nsplit) * w.ncols;
+    w.kb_begin = 0;
+    w.kb_end = p.k_blocks;
+    return true;
+  }
+  if (p.sk_per <= 0) return false;
   const int kb = p.k_blocks;
   const int u0 = pair_id * p.sk_per;
   const int u1 = min(u0 + p.sk_per, p.sk_units);
@@ -128,7 +149,7 @@ __device__ __forceinline__ bool pair_work_item(const GemmParams &p, int pair_id,
   const int t_rel = u0 / kb + (i - n_dp);
   if (t_rel * kb >= u1) return false;
   w.t_rel = t_rel;
-  w.tile = p.sk_tile0 + t_rel;
+  w.tile = p.dp_tiles + t_rel;
   w.kb_begin = max(u0 - t_rel * kb, 0);
   w.kb_end = min(u1 - t_rel * kb, kb);
   const int first = (t_rel * kb) / p.sk_per;
@@ -198,12 +219,14 @@ __device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const C
                                                     uint8_t *stage_buf, uint32_t &chunk_count,
                                                     int lane, int mode = kEpiNormal,
                                                     int32_t *slot = nullptr, int nparts = 0,
-                                                    int own_part = 0, int64_t part_stride = 0) {
+                                                    int own_part = 0, int64_t part_stride = 0,
+                                                    int ncols = COLS) {
   const int row = row0 + lane;
   const bool row_ok = row < p.M;
   const float sa = row_ok ? __ldg(p.s_a + row) : 0.0f;
-  // a warp whose 32 rows all lie past M has nothing to store
-  const int cols_here = row0 < p.M ? COLS : 0;
+  // a warp whose 32 rows all lie past M has nothing to store; a narrow tile
+  // (ncols < COLS, a multiple of 32) has fewer chunks
+  const int cols_here = row0 < p.M ? (ncols < COLS ? ncols : COLS) : 0;
 #pragma unroll 1
   for (int c = 0; c < cols_here; c += kEpiChunk) {
     const int col0 = col_base + c;
@@ -533,7 +556,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // leader's "full" barrier; the leader's commits arrive on "empty" and
 // accumulator-"full" barriers in both CTAs; both CTAs' epilogue warps arrive
 // on the leader's accumulator-"empty" barrier.
-constexpr int kPairBN = 256;
 
 template <int STAGES>
 struct PairLayout {
@@ -559,6 +581,7 @@ template <int STAGES, bool RAW_OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_i8_tcgen05_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                                 const __grid_constant__ CUtensorMap tmap_b,
+                                const __grid_constant__ CUtensorMap tmap_b_tail,
                                 const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
   using L = PairLayout<STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -592,6 +615,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     fence_mbarrier_init();
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
+    if (p.tail_nsplit > 1) tma_prefetch_desc(&tmap_b_tail);
     if constexpr (!RAW_OUT) tma_prefetch_desc(&tmap_y);
   }
   if (warp == 1) {
@@ -614,6 +638,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // preceding kernel (programmatic dependent launch); q after the wait.
       int prefetched = 0;
       WorkItem w;
+      // An item of ncols columns loads this CTA's ncols / 2 rows of Wq (the
+      // narrow tail tiles through their own, narrower TMA box).
+      auto b_map = [&](const WorkItem &it) { return it.ncols == kPairBN ? &tmap_b : &tmap_b_tail; };
+      auto b_row = [&](const WorkItem &it, int nb) {
+        return nb * kPairBN + it.n_off + static_cast<int>(rank) * (it.ncols / 2);
+      };
+      auto stage_tx = [&](const WorkItem &it) {
+        return 2u * static_cast<uint32_t>(L::kABytes + (it.ncols / 2) * kBK);
+      };
       if (pair_work_item(p, pair_id, num_pairs, 0, w)) {
         int mb0, nb0;
         pair_tile_coords(w.tile, p, mb0, nb0);
@@ -621,9 +654,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         prefetched = nkb < STAGES ? nkb : STAGES;
         for (int i = 0; i < prefetched; ++i) {
           uint8_t *sb = smem + i * L::kStageBytes + L::kABytes;
-          if (rank == 0) mbar_arrive_expect_tx(&full[i], 2 * L::kStageBytes);
-          tma_load_2d_pair(&tmap_b, map_to_cta(smem_addr(&full[i]), 0), sb,
-                           (w.kb_begin + i) * kBK, nb0 * kPairBN + static_cast<int>(rank) * 128);
+          if (rank == 0) mbar_arrive_expect_tx(&full[i], stage_tx(w));
+          tma_load_2d_pair(b_map(w), map_to_cta(smem_addr(&full[i]), 0), sb,
+                           (w.kb_begin + i) * kBK, b_row(w, nb0));
         }
       }
       grid_dependency_wait();
@@ -641,9 +674,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (prefetched > 0) {
             --prefetched;  // armed and Wq in flight already
           } else {
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::kStageBytes);
-            tma_load_2d_pair(&tmap_b, leader_full, sb, kb * kBK,
-                             nb * kPairBN + static_cast<int>(rank) * 128);
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], stage_tx(w));
+            tma_load_2d_pair(b_map(w), leader_full, sb, kb * kBK, b_row(w, nb));
           }
           tma_load_2d_pair(&tmap_a, leader_full, sa, kb * kBK, mb * 256 + static_cast<int>(rank) * 128);
           ++issued;
@@ -663,7 +695,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_i8(2 * kBM, kPairBN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -678,6 +709,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPairBN);
+        const uint32_t idesc = idesc_i8(2 * kBM, w.ncols);
         for (int kb = w.kb_begin; kb < w.kb_end; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             ok = false;
@@ -730,13 +762,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
+      // this warp: TMEM lane quarter `quarter`, columns [half * ncols / 2, +ncols / 2)
+      const int wcols = w.ncols / 2;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * kPairBN + half * (kPairBN / 2));
+                             static_cast<uint32_t>(acc * kPairBN + half * wcols);
       const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quarter * 32;
-      const int col_base = nb * kPairBN + half * (kPairBN / 2);
+      const int col_base = nb * kPairBN + w.n_off + half * wcols;
       if (w.nparts == 1) {
         epilogue_warp_slice<kPairBN / 2, RAW_OUT>(p, &tmap_y, t_row, row0, col_base, stage_buf,
-                                                  chunk_count, lane);
+                                                  chunk_count, lane, kEpiNormal, nullptr, 0, 0, 0,
+                                                  wcols);
       } else {
         // Shared-out tile: the last contribution to arrive finishes it.  The
         // part holding k-block 0 is this pair's last item and usually the
