@@ -199,8 +199,13 @@ class Layer:
             })
         self.x_host_bits = x_bits
         self.i = 0
-        self.variant = w8a8.select(M, N, K)["variant_name"]
-        self.launches_per_step = 1 if self.variant == "gemv" else 2
+        plan = w8a8.select(M, N, K)
+        self.variant = plan["variant_name"]
+        # GEMV: quantization in its prologue; CTA-pair GEMM with a full
+        # workspace: quantization inside the same launch when the plan says so
+        # (eager launches; under stream capture the layer takes two launches)
+        self.launches_per_step = 1 if (self.variant == "gemv" or
+                                       (plan["quant_in_gemm_launch"] and with_ws)) else 2
 
     def step(self):
         s = self.sets[self.i]

@@ -102,6 +102,10 @@ typedef struct {
     int32_t tail_tiles_nsplit; /* GEMM_PAIR: 2 when the tiles of the last,
                               partial round are cut along N into two
                               128-column tiles (one per pair); else 0 */
+    int32_t quant_in_gemm_launch; /* GEMM_PAIR: 1 when w8a8_linear_fused runs the
+                              per-token quantization inside the GEMM launch
+                              (given the full workspace, outside stream
+                              capture); else 0 */
 } w8a8_plan;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -142,10 +146,12 @@ W8A8_API int w8a8_quant_act(const void *x_bf16, int64_t M, int64_t K, int64_t ld
 
 /*
  * Scratch bytes for (M, N, K) on a 148-SM B200: w8a8_linear_fused's int8
- * activations and their scales, plus, when the plan shares its last tiles
- * out along K (w8a8_plan.split_tiles > 0), the int32 partial sums and arrival
- * counters of that region.  A workspace too small for the K-split region
- * still works: the layer then runs without the split (slower tail wave).
+ * activations and their scales, one 64-bit counter per 128 rows (the fused
+ * quantization's progress), plus, when the plan shares its last tiles out
+ * along K (w8a8_plan.split_tiles > 0), the int32 partial sums and arrival
+ * counters of that region.  Nothing in it needs initializing.  A workspace
+ * holding only q and s_a still works: the layer then runs as two launches
+ * and without the K split.
  */
 W8A8_API int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes);
 
@@ -183,8 +189,13 @@ W8A8_API int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_
  * intermediates (then they are used instead of workspace).
  * workspace: w8a8_workspace_size(M,N,K) bytes, 16-byte aligned (256
  * recommended).  Required: the bytes for q and s_a, unless both q_out and
- * s_a_out are given; the rest (the K-split region) is optional, see
- * w8a8_workspace_size.
+ * s_a_out are given.  The rest is optional: with the row-block counters that
+ * follow q and s_a, a plan on the CTA-pair GEMM quantizes x inside the GEMM
+ * launch itself (one launch; its producers wait only for the 128-row blocks
+ * they load, so the MMAs start while later rows are still being quantized);
+ * without them the call launches the quantization kernel and then the GEMM.
+ * Both give bit-identical results.  The K-split region comes last (see
+ * w8a8_workspace_size).
  */
 W8A8_API int w8a8_linear_fused(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
                       const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,
@@ -237,7 +248,7 @@ W8A8_API int w8a8_selftest_bounded_wait(int64_t limit_ns, w8a8_stream_t stream);
  * computes exactly what w8a8_linear_fused computes (same arguments minus
  * q_out / s_a_out / workspace), but keeps the int8 activations and their
  * scales in a scratch area compiled into the library: a static device array
- * of 16 MiB for q plus 64 KiB for the row scales.  Every GPU that loads this
+ * of 16 MiB for q plus 64 KiB for the row scales and 4 KiB of counters.  Every GPU that loads this
  * library holds that array until the process exits.
  *
  * Limits: M * K <= 16 MiB (16777216) and M <= 16384; a larger call returns

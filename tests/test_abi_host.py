@@ -243,3 +243,12 @@ def test_selector_is_total_and_consistent(M, KN):
     assert 1 <= p["grid"] <= 148
     if p["variant_name"] == "gemm_pair":
         assert tm == tn == 256 and p["grid"] % 2 == 0
+
+
+def test_quantization_inside_the_gemm_launch_plan():
+    # rows that fit one warp's registers and at most 4 passes of 8 rows per CTA
+    assert w8a8.select(4352, 9216, 3072)["quant_in_gemm_launch"] == 1
+    assert w8a8.select(4352, 12288, 3072)["quant_in_gemm_launch"] == 1
+    assert w8a8.select(4352, 3072, 12288)["quant_in_gemm_launch"] == 0   # K > 3072
+    assert w8a8.select(8704, 3072, 3072)["quant_in_gemm_launch"] == 0    # 8 passes
+    assert w8a8.select(100, 3072, 3072)["quant_in_gemm_launch"] == 0     # not the pair kernel

@@ -551,3 +551,55 @@ def test_pair_n_split_tail_exact(M, N, K, nsplit):
     assert np.array_equal(acc.cpu().numpy(), ref)
     y32, y_ref = oracle.epilogue(ref, s_a, s_w, b)
     assert check_y(bits_of(y), y_ref, y32, "n-split") == 0
+
+
+# ----------------------------------------------------------------- quantization fused into the GEMM launch
+
+def _fused_call(x, Wq, s_w, b, y, ws, ws_bytes, q_out=None, s_a_out=None):
+    st = B.w8a8_linear_fused(B._ptr(x), x.shape[0], x.shape[1], x.stride(0), B._ptr(Wq), B._ptr(s_w),
+                             B._ptr(b), Wq.shape[0], B._ptr(y), y.stride(0), B._ptr(q_out),
+                             B._ptr(s_a_out), B._ptr(ws), ws_bytes, B._stream())
+    assert st == 0, B.status_string(st)
+
+
+# (M, N, K, ldx): the QKV shape, a ragged M (last row block of 67 rows, last
+# pass of 3 rows per CTA group) with K = 3072, a short K (single-vector lanes)
+# and a strided x (ldx > K).
+FUSED_CASES = [(4352, 9216, 3072, 3072), (1091, 3072, 3072, 3072), (1537, 2048, 3072, 3200),
+               (2048, 2048, 512, 512)]
+
+
+@pytest.mark.parametrize("M,N,K,ldx", FUSED_CASES)
+def test_quantization_fused_into_pair_launch(M, N, K, ldx):
+    """With room for the row-block counters in the workspace, the pair plan
+    quantizes x inside the GEMM launch; the result must be bit-equal to the
+    two-launch path (workspace without the counters) and q, s_a must equal the
+    oracle's; y against the oracle on sampled rows."""
+    plan = w8a8.select(M, N, K)
+    assert plan["variant_name"] == "gemm_pair" and plan["quant_in_gemm_launch"] == 1
+    xb = synth.make_x(M, K, "studentt", 17)
+    x_full = np.zeros((M, ldx), np.uint16)
+    x_full[:, :K] = xb
+    x = to_dev(x_full)[:, :K]
+    w = synth.make_w(N, K, 17)
+    wq, sw = oracle.quantize_weights(w)
+    b = synth.make_bias(N, 17)
+    Wq, s_w, bd = torch.from_numpy(wq).cuda(), torch.from_numpy(sw).cuda(), to_dev(b)
+    need = w8a8.workspace_size(M, N, K)
+    ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+    q_head = ((M * K + 255) // 256) * 256 + ((4 * M + 255) // 256) * 256   # q and s_a only
+    y1 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    y3 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    s_a = torch.empty((M,), dtype=torch.float32, device="cuda")
+    _fused_call(x, Wq, s_w, bd, y1, ws, need)                    # one launch
+    _fused_call(x, Wq, s_w, bd, y2, ws, q_head)                  # quant kernel + GEMM
+    _fused_call(x, Wq, s_w, bd, y3, ws, need, q_out=q, s_a_out=s_a)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(y1.view(torch.int16), y3.view(torch.int16))
+    q_ref, s_ref = _quant_check(xb, q, s_a)
+    rows = sample_rows(M, seed=17, n_random=32)
+    y32, y_ref = oracle.epilogue(oracle.gemm_i32(q_ref[rows], wq), s_ref[rows], sw, b)
+    assert check_y(bits_of(y1)[rows], y_ref, y32, "fused launch") == 0

@@ -51,7 +51,7 @@ class Plan(ctypes.Structure):
                 ("tile_n", ctypes.c_int32), ("num_tiles", ctypes.c_int32),
                 ("grid", ctypes.c_int32), ("waves_x100", ctypes.c_int32),
                 ("split_tiles", ctypes.c_int32), ("split_kblocks_per_pair", ctypes.c_int32),
-                ("tail_tiles_nsplit", ctypes.c_int32)]
+                ("tail_tiles_nsplit", ctypes.c_int32), ("quant_in_gemm_launch", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {f: getattr(self, f) for f, _ in self._fields_}

@@ -88,6 +88,14 @@ int check_n(int64_t N, int64_t ldy) {
 
 // ---------------------------------------------------------------- selector
 
+// The fused pair launch quantizes x with its epilogue warps (8 per CTA), one
+// row per warp per pass, before they turn to the epilogues: used when a row
+// fits one warp's registers and at most kFuseMaxPasses passes are needed (more
+// would hold back the first epilogues long enough to stall the MMAs).
+constexpr int64_t kFuseMaxK = 3072;
+constexpr int64_t kFuseMaxPasses = 4;
+
+
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 inline bool gemv_fits(int64_t M, int64_t K, int max_smem) {
@@ -175,6 +183,8 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     plan->tile_n = 256;
     plan->num_tiles = static_cast<int32_t>(tiles);
     plan->grid = static_cast<int32_t>(2 * pairs);
+    plan->quant_in_gemm_launch =
+        (K <= kFuseMaxK && cdiv(M, 2 * pairs * kEpiWarps) <= kFuseMaxPasses) ? 1 : 0;
     if (nsplit > 1) {
       plan->tail_tiles_nsplit = static_cast<int32_t>(nsplit);
       plan->waves_x100 = static_cast<int32_t>(100 * full + 100 / nsplit);
@@ -202,6 +212,12 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
 // ---------------------------------------------------------------- workspace
 
 size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+// Per-128-row-block "rows quantized" counters of the fused pair launch.
+size_t ready_counter_bytes(int64_t M) {
+  return align256(static_cast<size_t>(cdiv(M, kBM)) * sizeof(unsigned long long));
+}
+
 
 size_t fused_workspace_bytes(int64_t M, int64_t K) {
   return align256(static_cast<size_t>(M) * static_cast<size_t>(K)) +
@@ -425,11 +441,19 @@ int launch_gemm_t(const w8a8_plan &plan, const int8_t *q, const float *s_a, int6
                    mb, my, p);
 }
 
-template <bool RAW>
+// The per-token quantization fused into the pair launch: x is quantized into
+// q / s_a (the GEMM's operands) by the kernel itself.
+struct FuseArgs {
+  const void *x;
+  int64_t ldx;
+  unsigned long long *row_ready;  // cdiv(M, 128) counters
+};
+
+template <bool RAW, bool FUSE>
 int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, int64_t M,
                      int64_t K, const int8_t *wq, const float *s_w, const void *bias, int64_t N,
                      void *y, int64_t ldy, int32_t *acc, const SplitRegion &split,
-                     cudaStream_t stream) {
+                     const FuseArgs *fuse, cudaStream_t stream) {
   using L = PairLayout<kGemmStagesPair>;
   CUtensorMap ma, mb, mbt, my;
   int st = encode_i8_map(&ma, q, M, K, kBM);
@@ -487,7 +511,22 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
   } else if (plan.split_tiles > 0 && plan.num_tiles < plan.grid / 2) {
     grid = 2 * plan.num_tiles;  // unsplit and under one wave: one pair per tile
   }
-  constexpr auto kernel = gemm_i8_tcgen05_pair_kernel<kGemmStagesPair, RAW>;
+  p.x = nullptr;
+  p.ldx = 0;
+  p.q_w = nullptr;
+  p.s_a_w = nullptr;
+  p.row_ready = nullptr;
+  p.fuse_tag = 0;
+  if (FUSE) {
+    p.x = static_cast<const uint16_t *>(fuse->x);
+    p.ldx = fuse->ldx;
+    p.q_w = const_cast<int8_t *>(q);
+    p.s_a_w = const_cast<float *>(s_a);
+    p.row_ready = fuse->row_ready;
+    p.fuse_tag = g_split_epoch.fetch_add(1, std::memory_order_relaxed) & ((1ull << 48) - 1);
+    if (p.fuse_tag == 0) p.fuse_tag = 1;
+  }
+  constexpr auto kernel = gemm_i8_tcgen05_pair_kernel<kGemmStagesPair, RAW, FUSE>;
   st = ensure_smem_limit<kernel>(L::kSmemBytes);
   if (st != W8A8_OK) return st;
   return launch_ex(true, kernel, dim3(grid), dim3(kGemmThreads), L::kSmemBytes, stream, ma, mb,
@@ -586,10 +625,10 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
   }
   if (plan.variant == W8A8_VARIANT_GEMM_PAIR) {
     const SplitRegion split = split_region(plan, split_ws, split_ws_bytes);
-    return acc ? launch_gemm_pair<true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc, split,
-                                        stream)
-               : launch_gemm_pair<false>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc,
-                                         split, stream);
+    return acc ? launch_gemm_pair<true, false>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc,
+                                               split, nullptr, stream)
+               : launch_gemm_pair<false, false>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc,
+                                                split, nullptr, stream);
   }
   if (plan.variant == W8A8_VARIANT_GEMM_BN128) {
     return acc ? launch_gemm_t<128, kGemmStages128, true>(plan, q, s_a, M, K, Wq, s_w, bias, N,
@@ -605,13 +644,14 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
 
 // ---------------------------------------------------------------- static scratch
 // Scratch for w8a8_linear_fused_noalloc: the int8 activations (up to 16 MiB)
-// followed by their fp32 row scales (up to 16384 rows).  In host code the
+// followed by their fp32 row scales (up to 16384 rows) and 4 KiB for the
+// fused launch's row-block counters.  In host code the
 // array's name only stands in for the device object; its device address is
 // looked up once per device with cudaGetSymbolAddress.
 constexpr size_t kNoAllocMaxQBytes = static_cast<size_t>(16) << 20;
 constexpr int64_t kNoAllocMaxRows = 16384;
 constexpr size_t kNoAllocScratchBytes =
-    kNoAllocMaxQBytes + static_cast<size_t>(kNoAllocMaxRows) * sizeof(float);
+    kNoAllocMaxQBytes + static_cast<size_t>(kNoAllocMaxRows) * sizeof(float) + 4096;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 struct NoAllocScratch {
@@ -733,7 +773,8 @@ int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes) {
   if (st != W8A8_OK) return st;
   *bytes = plan.variant == W8A8_VARIANT_GEMV
                ? 0
-               : fused_workspace_bytes(M, K) + split_workspace_bytes(plan);
+               : fused_workspace_bytes(M, K) + ready_counter_bytes(M) +
+                     split_workspace_bytes(plan);
   return W8A8_OK;
 }
 
@@ -792,7 +833,7 @@ int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const in
     return launch_gemv_m<true, false>(plan, p, d->max_smem_optin, d->sms, stream);
   }
 
-  // workspace layout: [q (M*K) | s_a (M floats) | K-split region]
+  // workspace layout: [q (M*K) | s_a (M floats) | row-ready counters | K-split region]
   int8_t *q = q_out;
   float *s_a = s_a_out;
   const size_t qs_bytes = fused_workspace_bytes(M, K);
@@ -802,11 +843,34 @@ int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const in
     if (!q) q = reinterpret_cast<int8_t *>(ws);
     if (!s_a) s_a = reinterpret_cast<float *>(ws + align256(static_cast<size_t>(M * K)));
   }
+  const size_t head = qs_bytes + ready_counter_bytes(M);
+  const bool have_ready = workspace && aligned16(workspace) && ws_bytes >= head;
   void *split_ws = nullptr;
   size_t split_bytes = 0;
-  if (workspace && ws_bytes > qs_bytes && aligned16(workspace)) {
-    split_ws = static_cast<uint8_t *>(workspace) + qs_bytes;
-    split_bytes = ws_bytes - qs_bytes;
+  if (have_ready && ws_bytes > head) {
+    split_ws = static_cast<uint8_t *>(workspace) + head;
+    split_bytes = ws_bytes - head;
+  }
+  // The fused launch tags its row flags with a value drawn here, on the host:
+  // a captured graph would replay one tag, so under stream capture the two
+  // launches are used instead.
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  if (plan.variant == W8A8_VARIANT_GEMM_PAIR && plan.quant_in_gemm_launch && have_ready &&
+      capture == cudaStreamCaptureStatusNone) {
+    // one launch: the pair kernel quantizes x itself, its producers waiting
+    // only for the 128-row blocks they load
+    FuseArgs f;
+    f.x = x;
+    f.ldx = ldx;
+    f.row_ready = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) +
+                                                         qs_bytes);
+    const SplitRegion split = split_region(plan, split_ws, split_bytes);
+    return launch_gemm_pair<false, true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, nullptr,
+                                         split, &f, stream);
   }
   st = launch_quant(x, M, K, ldx, q, s_a, stream);
   if (st != W8A8_OK) return st;

@@ -37,6 +37,7 @@
 #include <cstdint>
 
 #include "w8a8_ptx.cuh"
+#include "w8a8_quant.cuh"
 
 namespace w8a8 {
 
@@ -95,6 +96,21 @@ struct GemmParams {
   // memory needs no clearing; the electing contribution resets it to 0.
   unsigned long long *split_counters;
   unsigned long long split_epoch;  // 1 .. 2^56 - 1
+  // CTA-pair kernel with the per-token quantization fused in (K <= 3072: a
+  // row fits one warp's registers): the epilogue warps of all CTAs first
+  // quantize the rows of x (bf16 [M, K], row stride ldx) into q_w / s_a_w --
+  // the buffers the GEMM then reads through tmap_a and s_a.  In pass j, CTA c
+  // takes rows 8 c .. 8 c + 7 + j * 8 * gridDim.x (one per epilogue warp), so
+  // the 128-row blocks complete in order; after each pass one thread of the
+  // CTA adds its rows to the block's counter, (fuse_tag << 16) | rows (a
+  // counter holding another launch's tag counts as 0: nothing needs
+  // clearing).  A producer waits for its block's count before loading q.
+  const uint16_t *x;
+  int64_t ldx;
+  int8_t *q_w;
+  float *s_a_w;
+  unsigned long long *row_ready;   // cdiv(M, 128) counters
+  unsigned long long fuse_tag;     // 1 .. 2^48 - 1
 };
 
 constexpr unsigned long long kSplitEpochMask = (1ull << 56) - 1;
@@ -159,19 +175,53 @@ __device__ __forceinline__ bool pair_work_item(const GemmParams &p, int pair_id,
   return true;
 }
 
-// Registers one arrival on a K-split counter for launch tag `epoch`; returns
-// how many contributions had arrived before (-1 if the retry bound ran out,
-// which also sets the device error word).
-__device__ __forceinline__ int split_arrive(unsigned long long *counter, unsigned long long epoch) {
+// Registers one arrival on a tagged counter, (tag << BITS) | arrivals, for
+// launch tag `tag` (a counter holding another tag counts as 0); returns how
+// many arrivals came before (-1 if the retry bound ran out, which also sets
+// the device error word).
+template <int BITS>
+__device__ __forceinline__ int tagged_arrive(unsigned long long *counter, unsigned long long tag,
+                                             unsigned long long add = 1) {
+  constexpr unsigned long long kMask = (1ull << BITS) - 1;
   unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(counter);
   for (int i = 0; i < (1 << 20); ++i) {
-    const unsigned long long before = (cur >> 8) == epoch ? (cur & 0xFFull) : 0ull;
-    const unsigned long long prev = atomicCAS(counter, cur, (epoch << 8) | (before + 1ull));
+    const unsigned long long before = (cur >> BITS) == tag ? (cur & kMask) : 0ull;
+    const unsigned long long prev = atomicCAS(counter, cur, (tag << BITS) | (before + add));
     if (prev == cur) return static_cast<int>(before);
     cur = prev;
   }
   atomicOr(&g_device_error, W8A8_DEVERR_TIMEOUT);
   return -1;
+}
+
+__device__ __forceinline__ int split_arrive(unsigned long long *counter, unsigned long long epoch) {
+  return tagged_arrive<8>(counter, epoch);
+}
+
+// Waits (acquire, bounded like every other wait) until the rows of 128-row
+// block b of q are quantized; then their q and s_a may be read (the TMA
+// loads that follow included).
+__device__ __forceinline__ bool rows_block_wait(const GemmParams &p, int b,
+                                                volatile int *abort_flag) {
+  const int r0 = b * kBM;
+  const int n = p.M - r0 < kBM ? p.M - r0 : kBM;
+  const unsigned long long want = (p.fuse_tag << 16) | static_cast<unsigned long long>(n);
+  const unsigned long long *c = p.row_ready + b;
+  if (ld_acquire_gpu_u64(c) != want) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1; ld_acquire_gpu_u64(c) != want; ++i) {
+      if ((i & 15u) == 0u) {
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          atomicOr(&g_device_error, W8A8_DEVERR_TIMEOUT);
+          return false;
+        }
+      }
+    }
+  }
+  fence_proxy_async_global();  // order the TMA reads after the acquire
+  return true;
 }
 
 // Partial-sum slice of pair `pair` on shared-out tile t_rel.  Slot t_rel +
@@ -223,7 +273,9 @@ __device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const C
                                                     int ncols = COLS) {
   const int row = row0 + lane;
   const bool row_ok = row < p.M;
-  const float sa = row_ok ? __ldg(p.s_a + row) : 0.0f;
+  // s_a may have been written earlier in this same launch (fused
+  // quantization): read it through L2, never the non-coherent path
+  const float sa = row_ok ? __ldcg(p.s_a + row) : 0.0f;
   // a warp whose 32 rows all lie past M has nothing to store; a narrow tile
   // (ncols < COLS, a multiple of 32) has fewer chunks
   const int cols_here = row0 < p.M ? (ncols < COLS ? ncols : COLS) : 0;
@@ -577,7 +629,7 @@ __device__ __forceinline__ void pair_tile_coords(int t, const GemmParams &p, int
   gemm_tile_coords(t, p, mb, nb);  // p.num_m_blk counts 256-row blocks here
 }
 
-template <int STAGES, bool RAW_OUT>
+template <int STAGES, bool RAW_OUT, bool FUSE_QUANT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_i8_tcgen05_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                                 const __grid_constant__ CUtensorMap tmap_b,
@@ -660,9 +712,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
       }
       grid_dependency_wait();
+      int ready_blk = -1;  // fused quantization: the q block known to be complete
       for (int it = 0; ok && pair_work_item(p, pair_id, num_pairs, it, w); ++it) {
         int mb, nb;
         pair_tile_coords(w.tile, p, mb, nb);
+        if constexpr (FUSE_QUANT) {
+          const int blk = mb * 2 + static_cast<int>(rank);
+          if (blk != ready_blk && blk * kBM < p.M) {
+            if (!rows_block_wait(p, blk, abort_flag)) {
+              ok = false;
+              break;
+            }
+            ready_blk = blk;
+          }
+        }
         for (int kb = w.kb_begin; kb < w.kb_end; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -752,11 +815,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     const int slice = static_cast<int>(rank) * kEpiWarps + e;
-    grid_dependency_wait();  // s_a comes from the preceding kernel
+    grid_dependency_wait();  // s_a (or, fused, x) comes from the preceding kernel
+    if constexpr (FUSE_QUANT) {
+      // pass j: this CTA's 8 rows 8 c + j * 8 * gridDim.x + e (one 128-row
+      // block: 8 divides 128), then one arrival for all of them
+      const int stride = static_cast<int>(gridDim.x) * kEpiWarps;
+      for (int base = static_cast<int>(blockIdx.x) * kEpiWarps; base < p.M; base += stride) {
+        const int row = base + e;
+        if (row < p.M)
+          quant_row_by_warp<12>(p.x + static_cast<int64_t>(row) * p.ldx, p.K,
+                                p.q_w + static_cast<int64_t>(row) * p.K, p.s_a_w + row, lane);
+        fence_proxy_async_global();
+        __threadfence();  // release: every lane's q and s_a stores before the count
+        named_barrier_sync(1, kEpiWarps * 32);
+        if (e == 0 && lane == 0) {
+          const int rows = p.M - base < kEpiWarps ? p.M - base : kEpiWarps;
+          tagged_arrive<16>(&p.row_ready[base / kBM], p.fuse_tag,
+                            static_cast<unsigned long long>(rows));
+        }
+      }
+    }
     WorkItem w;
     for (int it = 0; pair_work_item(p, pair_id, num_pairs, it, w); ++it) {
       int mb, nb;
       pair_tile_coords(w.tile, p, mb, nb);
+      if constexpr (FUSE_QUANT) {  // acquire this slice's rows (their s_a)
+        const int blk = mb * 2 + static_cast<int>(rank);
+        if (lane == 0 && blk * kBM < p.M) rows_block_wait(p, blk, abort_flag);
+        __syncwarp();
+      }
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], acc_phase, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);

@@ -121,6 +121,52 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v, int width) {
   return v;
 }
 
+// One warp quantizes one row of K elements (K % 8 == 0) into qr / *s_out.
+// Rows of up to 32 x V vectors of 8 stay in registers (x read once); longer
+// rows take two passes, max |x| first, then the codes (the second pass reading
+// the row back from L2).  All 32 lanes must call it.
+template <int V>
+__device__ __forceinline__ void quant_row_by_warp(const uint16_t *__restrict__ xr, int K,
+                                                  int8_t *__restrict__ qr, float *s_out,
+                                                  int lane) {
+  const int nvec = K >> 3;
+  const uint4 *xv = reinterpret_cast<const uint4 *>(xr);
+  uint2 *qv = reinterpret_cast<uint2 *>(qr);
+  if (nvec <= 32 * V) {
+    uint4 v[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const int vi = lane + 32 * j;
+      v[j] = vi < nvec ? __ldcs(xv + vi) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      if (j & 1) m1 = absmax_vec8(v[j], m1); else m0 = absmax_vec8(v[j], m0);
+    }
+    const float amax = __uint_as_float(warp_max_u32(__float_as_uint(fmaxf(m0, m1)), 32));
+    const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+    const bool fast = quant_fast_ok(sc);
+    const float rc = fast ? __frcp_rn(sc) : 0.0f;
+    if (lane == 0) *s_out = sc;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const int vi = lane + 32 * j;
+      if (vi < nvec) qv[vi] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(v[j], sc, rc, fast);
+    }
+  } else {
+    float m = 0.0f;
+    for (int vi = lane; vi < nvec; vi += 32) m = absmax_vec8(__ldg(xv + vi), m);
+    const float amax = __uint_as_float(warp_max_u32(__float_as_uint(m), 32));
+    const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+    const bool fast = quant_fast_ok(sc);
+    const float rc = fast ? __frcp_rn(sc) : 0.0f;
+    if (lane == 0) *s_out = sc;
+    for (int vi = lane; vi < nvec; vi += 32)
+      qv[vi] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(__ldcs(xv + vi), sc, rc, fast);
+  }
+}
+
 // Very long rows (K > 24576): one block of 256 threads per row, two passes
 // over the row -- max |x| first, then quantize -- the second pass reading the
 // row back from L2.
