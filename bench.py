@@ -201,11 +201,9 @@ class Layer:
         self.i = 0
         plan = w8a8.select(M, N, K)
         self.variant = plan["variant_name"]
-        # GEMV: quantization in its prologue; CTA-pair GEMM with a full
-        # workspace: quantization inside the same launch when the plan says so
-        # (eager launches; under stream capture the layer takes two launches)
-        self.launches_per_step = 1 if (self.variant == "gemv" or
-                                       (plan["quant_in_gemm_launch"] and with_ws)) else 2
+        # GEMV: quantization in its prologue (one launch); GEMMs: the
+        # quantization kernel, then the GEMM
+        self.launches_per_step = 1 if self.variant == "gemv" else 2
 
     def step(self):
         s = self.sets[self.i]

@@ -102,10 +102,10 @@ typedef struct {
     int32_t tail_tiles_nsplit; /* GEMM_PAIR: 2 when the tiles of the last,
                               partial round are cut along N into two
                               128-column tiles (one per pair); else 0 */
-    int32_t quant_in_gemm_launch; /* GEMM_PAIR: 1 when w8a8_linear_fused runs the
-                              per-token quantization inside the GEMM launch
-                              (given the full workspace, outside stream
-                              capture); else 0 */
+    int32_t quant_in_gemm_launch; /* GEMM_PAIR: 1 when w8a8_linear_fused_ex
+                              with W8A8_FUSED_ONE_LAUNCH can run the per-token
+                              quantization inside the GEMM launch (given the
+                              full workspace, outside stream capture); else 0 */
 } w8a8_plan;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -146,12 +146,12 @@ W8A8_API int w8a8_quant_act(const void *x_bf16, int64_t M, int64_t K, int64_t ld
 
 /*
  * Scratch bytes for (M, N, K) on a 148-SM B200: w8a8_linear_fused's int8
- * activations and their scales, one 64-bit counter per 128 rows (the fused
- * quantization's progress), plus, when the plan shares its last tiles out
- * along K (w8a8_plan.split_tiles > 0), the int32 partial sums and arrival
- * counters of that region.  Nothing in it needs initializing.  A workspace
- * holding only q and s_a still works: the layer then runs as two launches
- * and without the K split.
+ * activations and their scales, one 64-bit counter per 128 rows (used by
+ * the one-launch option of w8a8_linear_fused_ex), plus, when the plan shares
+ * its last tiles out along K (w8a8_plan.split_tiles > 0), the int32 partial
+ * sums and arrival counters of that region.  Nothing in it needs
+ * initializing.  A workspace holding only q and s_a still works: the layer
+ * then runs without the K split.
  */
 W8A8_API int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes);
 
@@ -189,18 +189,34 @@ W8A8_API int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_
  * intermediates (then they are used instead of workspace).
  * workspace: w8a8_workspace_size(M,N,K) bytes, 16-byte aligned (256
  * recommended).  Required: the bytes for q and s_a, unless both q_out and
- * s_a_out are given.  The rest is optional: with the row-block counters that
- * follow q and s_a, a plan on the CTA-pair GEMM quantizes x inside the GEMM
- * launch itself (one launch; its producers wait only for the 128-row blocks
- * they load, so the MMAs start while later rows are still being quantized);
- * without them the call launches the quantization kernel and then the GEMM.
- * Both give bit-identical results.  The K-split region comes last (see
- * w8a8_workspace_size).
+ * s_a_out are given; the rest (row-block counters, K-split region) is
+ * optional, see w8a8_workspace_size.  Two launches: the quantization kernel,
+ * then the GEMM as a programmatic dependent launch.
  */
 W8A8_API int w8a8_linear_fused(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
                       const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,
                       void *y_bf16, int64_t ldy, int8_t *q_out_or_null, float *s_a_out_or_null,
                       void *workspace, size_t ws_bytes, w8a8_stream_t stream);
+
+/* Options of w8a8_linear_fused_ex. */
+#define W8A8_FUSED_ONE_LAUNCH 1  /* quantize inside the GEMM launch when the plan
+                                    allows it (w8a8_plan.quant_in_gemm_launch) */
+
+/*
+ * w8a8_linear_fused with options.  W8A8_FUSED_ONE_LAUNCH: on a CTA-pair plan
+ * with quant_in_gemm_launch set, a workspace holding the row-block counters
+ * (w8a8_workspace_size bytes) and a stream that is not capturing, the pair
+ * kernel quantizes x itself: the epilogue warps of all CTAs quantize the rows
+ * in row-block order before turning to the epilogues, and each producer waits
+ * only for the 128-row block it loads.  One launch instead of two,
+ * bit-identical results; on a B200 it measured 6-17% slower than the two
+ * launches, so it is not the default.  Otherwise the call is exactly
+ * w8a8_linear_fused.  Unknown option bits: W8A8_ERR_INVALID_ARG.
+ */
+W8A8_API int w8a8_linear_fused_ex(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
+                      const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,
+                      void *y_bf16, int64_t ldy, int8_t *q_out_or_null, float *s_a_out_or_null,
+                      void *workspace, size_t ws_bytes, int options, w8a8_stream_t stream);
 
 /*
  * End-to-end form of w8a8_linear_fused for callers holding HOST buffers:

@@ -555,10 +555,11 @@ def test_pair_n_split_tail_exact(M, N, K, nsplit):
 
 # ----------------------------------------------------------------- quantization fused into the GEMM launch
 
-def _fused_call(x, Wq, s_w, b, y, ws, ws_bytes, q_out=None, s_a_out=None):
-    st = B.w8a8_linear_fused(B._ptr(x), x.shape[0], x.shape[1], x.stride(0), B._ptr(Wq), B._ptr(s_w),
-                             B._ptr(b), Wq.shape[0], B._ptr(y), y.stride(0), B._ptr(q_out),
-                             B._ptr(s_a_out), B._ptr(ws), ws_bytes, B._stream())
+def _fused_call(x, Wq, s_w, b, y, ws, ws_bytes, q_out=None, s_a_out=None, options=0):
+    st = B.w8a8_linear_fused_ex(B._ptr(x), x.shape[0], x.shape[1], x.stride(0), B._ptr(Wq),
+                                B._ptr(s_w), B._ptr(b), Wq.shape[0], B._ptr(y), y.stride(0),
+                                B._ptr(q_out), B._ptr(s_a_out), B._ptr(ws), ws_bytes, options,
+                                B._stream())
     assert st == 0, B.status_string(st)
 
 
@@ -571,10 +572,10 @@ FUSED_CASES = [(4352, 9216, 3072, 3072), (1091, 3072, 3072, 3072), (1537, 2048, 
 
 @pytest.mark.parametrize("M,N,K,ldx", FUSED_CASES)
 def test_quantization_fused_into_pair_launch(M, N, K, ldx):
-    """With room for the row-block counters in the workspace, the pair plan
-    quantizes x inside the GEMM launch; the result must be bit-equal to the
-    two-launch path (workspace without the counters) and q, s_a must equal the
-    oracle's; y against the oracle on sampled rows."""
+    """With the one-launch option and room for the row-block counters, the
+    pair plan quantizes x inside the GEMM launch; the result must be bit-equal
+    to the two-launch path and q, s_a must equal the oracle's; y against the
+    oracle on sampled rows."""
     plan = w8a8.select(M, N, K)
     assert plan["variant_name"] == "gemm_pair" and plan["quant_in_gemm_launch"] == 1
     xb = synth.make_x(M, K, "studentt", 17)
@@ -593,9 +594,10 @@ def test_quantization_fused_into_pair_launch(M, N, K, ldx):
     y3 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     q = torch.empty((M, K), dtype=torch.int8, device="cuda")
     s_a = torch.empty((M,), dtype=torch.float32, device="cuda")
-    _fused_call(x, Wq, s_w, bd, y1, ws, need)                    # one launch
-    _fused_call(x, Wq, s_w, bd, y2, ws, q_head)                  # quant kernel + GEMM
-    _fused_call(x, Wq, s_w, bd, y3, ws, need, q_out=q, s_a_out=s_a)
+    one = B.FUSED_ONE_LAUNCH
+    _fused_call(x, Wq, s_w, bd, y1, ws, need, options=one)       # one launch
+    _fused_call(x, Wq, s_w, bd, y2, ws, q_head, options=one)     # no counters: two launches
+    _fused_call(x, Wq, s_w, bd, y3, ws, need, q_out=q, s_a_out=s_a, options=one)
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     assert torch.equal(y1.view(torch.int16), y3.view(torch.int16))

@@ -74,6 +74,8 @@ _SIGNATURES = {
                         _sz, _vp], _int),
     "w8a8_linear_fused": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp,
                            _vp, _sz, _vp], _int),
+    "w8a8_linear_fused_ex": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp,
+                              _vp, _sz, _int, _vp], _int),
     "w8a8_linear_fused_host": ([_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _sz,
                                 _vp], _int),
     "w8a8_linear_fused_noalloc": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp],
@@ -158,6 +160,15 @@ def w8a8_linear_fused(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, q_out, s_a_out, wo
                       ws_bytes, stream) -> int:
     return lib().w8a8_linear_fused(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, q_out, s_a_out,
                                    workspace, ws_bytes, stream)
+
+
+def w8a8_linear_fused_ex(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, q_out, s_a_out, workspace,
+                         ws_bytes, options, stream) -> int:
+    return lib().w8a8_linear_fused_ex(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, q_out, s_a_out,
+                                      workspace, ws_bytes, options, stream)
+
+
+FUSED_ONE_LAUNCH = 1
 
 
 def w8a8_linear_fused_host(x_host, M, K, Wq, s_w, bias, N, y_host, x_dev, y_dev, workspace,

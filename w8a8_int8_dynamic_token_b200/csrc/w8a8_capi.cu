@@ -799,6 +799,15 @@ int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const in
                       const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
                       int8_t *q_out, float *s_a_out, void *workspace, size_t ws_bytes,
                       w8a8_stream_t stream_) {
+  return w8a8_linear_fused_ex(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, q_out, s_a_out, workspace,
+                              ws_bytes, 0, stream_);
+}
+
+int w8a8_linear_fused_ex(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t *Wq,
+                         const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
+                         int8_t *q_out, float *s_a_out, void *workspace, size_t ws_bytes,
+                         int options, w8a8_stream_t stream_) {
+  if (options & ~W8A8_FUSED_ONE_LAUNCH) return W8A8_ERR_INVALID_ARG;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!x || !Wq || !s_w || !y) return W8A8_ERR_INVALID_ARG;
   int st = check_mk(M, K, ldx);
@@ -851,16 +860,18 @@ int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const in
     split_ws = static_cast<uint8_t *>(workspace) + head;
     split_bytes = ws_bytes - head;
   }
-  // The fused launch tags its row flags with a value drawn here, on the host:
-  // a captured graph would replay one tag, so under stream capture the two
+  // One launch only on request: measured slower than the two launches (the
+  // epilogue warps alone quantize with too little memory parallelism; see the
+  // design notes).  Its counters carry a tag drawn here, on the host: a
+  // captured graph would replay one tag, so under stream capture the two
   // launches are used instead.
   cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess) {
+  if ((options & W8A8_FUSED_ONE_LAUNCH) && cudaStreamIsCapturing(stream, &capture) != cudaSuccess) {
     cudaGetLastError();
     return W8A8_ERR_CUDA;
   }
-  if (plan.variant == W8A8_VARIANT_GEMM_PAIR && plan.quant_in_gemm_launch && have_ready &&
-      capture == cudaStreamCaptureStatusNone) {
+  if ((options & W8A8_FUSED_ONE_LAUNCH) && plan.variant == W8A8_VARIANT_GEMM_PAIR &&
+      plan.quant_in_gemm_launch && have_ready && capture == cudaStreamCaptureStatusNone) {
     // one launch: the pair kernel quantizes x itself, its producers waiting
     // only for the 128-row blocks they load
     FuseArgs f;
