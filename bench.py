@@ -152,18 +152,30 @@ def profile_traffic(kernel_tag: str):
     h = re.search(r"source_sha256:\s*([0-9a-f]{16,64})", text)
     if not m:
         return None, None
-    if h and h.group(1) != kernel_source_hash()[: len(h.group(1))]:
+    if h and h.group(1) != kernel_source_hash(kernel_tag)[: len(h.group(1))]:
         return None, "stale"
     return float(m.group(1)), "ncu"
 
 
-def kernel_source_hash() -> str:
+# The device source files each profiled kernel is built from.
+KERNEL_SOURCES = {
+    "gemm_i8_tcgen05": ("w8a8_gemm.cuh", "w8a8_ptx.cuh", "w8a8_quant.cuh"),
+    "gemv_i8": ("w8a8_gemv.cuh", "w8a8_ptx.cuh", "w8a8_quant.cuh"),
+    "quant_rows": ("w8a8_quant.cuh", "w8a8_ptx.cuh"),
+}
+
+
+def kernel_source_hash(kernel_tag: str = "") -> str:
+    """sha256 of the device sources of the kernel a profile tag names (all of
+    them for an unknown tag)."""
     d = os.path.join(ROOT, "w8a8_int8_dynamic_token_b200", "csrc")
+    names = next((v for k, v in KERNEL_SOURCES.items() if kernel_tag.startswith(k)), None)
+    if names is None:
+        names = [n for n in os.listdir(d) if n.endswith((".cu", ".cuh"))]
     hs = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(d, name), "rb") as f:
-                hs.update(f.read())
+    for name in sorted(names):
+        with open(os.path.join(d, name), "rb") as f:
+            hs.update(f.read())
     return hs.hexdigest()
 
 
@@ -513,7 +525,56 @@ def extra_components(args, dev, dist, peaks, world):
         del layers, up, down
         torch.cuda.empty_cache()
         out["dit_block"] = dit_block_component(dev, dist, max(10, steps // 4))
+        out["small_m"] = small_m_component(dev, dist, peaks, steps)
+        out["unpack_int32_weights"] = unpack_component(dev, dist, peaks, steps)
     return out
+
+
+def small_m_component(dev, dist, peaks, steps):
+    """The selector's small-M regime on the QKV weight (K = 3072, N = 9216):
+    whole layer per M, with the kernel chosen, TOPS and the weight-stream
+    bandwidth (these layers are bound by reading Wq once)."""
+    res = {}
+    for M in (16, 17, 64, 128, 256, 512, 1024):
+        case = synth.LayerCase(f"qkv_m{M}", M, 3072, 9216, "studentt", 0)
+        L = Layer(case, dev)
+        t = timed(L.step, steps, 5, dist, graph=True) / steps
+        algo = 2 * M * case.K + case.N * case.K + 6 * case.N + 2 * M * case.N
+        res[f"M={M}"] = {"us": round(t * 1e6, 2), "variant": L.variant,
+                         "TOPS": round(case.ops / t / 1e12, 1),
+                         "GBs": round(algo / t / 1e9, 1),
+                         "frac_hbm": round(algo / t / 1e9 / peaks["hbm_gbs"], 4)}
+        del L
+        torch.cuda.empty_cache()
+    res["timing"] = "CUDA graph of back-to-back layer calls, inputs rotated over > 2x L2"
+    return res
+
+
+def unpack_component(dev, dist, peaks, steps):
+    """Loading packed int32 weight storage (four codes biased by 128 per word)
+    into the GEMM's int8 layout: the AdaLN weight, 18432 x 3072."""
+    import w8a8_int8_dynamic_token_b200 as w8a8
+    N, K = 18432, 3072
+    nsets = n_sets(2 * N * K)
+    packed = [torch.randint(-2**31, 2**31 - 1, (N, K // 4), dtype=torch.int32, device=dev)
+              for _ in range(nsets)]
+    outs = [torch.empty((N, K), dtype=torch.int8, device=dev) for _ in range(nsets)]
+    B = w8a8.binding
+    i = [0]
+
+    def step():
+        j = i[0] % nsets
+        i[0] += 1
+        st = B.w8a8_unpack_int32_weights(B._ptr(packed[j]), N, K, B._ptr(outs[j]), B._stream())
+        if st != 0:
+            raise RuntimeError(B.status_string(st))
+
+    t = timed(step, steps, 5, dist, graph=True) / steps
+    gbs = 2 * N * K / t / 1e9
+    del packed, outs
+    torch.cuda.empty_cache()
+    return {"us": round(t * 1e6, 2), "GBs": round(gbs, 1),
+            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_launch": 2 * N * K}
 
 
 def dit_block_component(dev, dist, steps):

@@ -82,7 +82,9 @@ typedef enum {
     W8A8_VARIANT_GEMV = 1,          /* M <= 16: CUDA-core int8 dot products */
     W8A8_VARIANT_GEMM_BN128 = 2,    /* tcgen05 kind::i8, 128x128 tiles */
     W8A8_VARIANT_GEMM_BN256 = 3,    /* tcgen05 kind::i8, 128x256 tiles */
-    W8A8_VARIANT_GEMM_PAIR = 4      /* tcgen05 kind::i8 on CTA pairs, 256x256 tiles */
+    W8A8_VARIANT_GEMM_PAIR = 4,     /* tcgen05 kind::i8 on CTA pairs, 256x256 tiles */
+    W8A8_VARIANT_GEMM_BN64 = 5      /* tcgen05 kind::i8, 128x64 tiles (small M: more
+                                       CTAs streaming the weights) */
 } w8a8_variant;
 
 /* The selector's decision for one (M, N, K); see w8a8_select. */

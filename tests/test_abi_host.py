@@ -98,12 +98,25 @@ def _golden(name):
 
 
 def test_selector_small_m_goes_to_gemv():
+    # The AdaLN modulation layer runs at M = batch (1, or 2 with CFG), below
+    # the 16 rows a torch._int_mm path cannot serve: every such M is served
+    # here, by the GEMV up to 4 rows (measured crossover) and by the tcgen05
+    # GEMM above.
     g = _golden("int_mm_min_rows.txt")
     lim, K, N = g["int_mm_min_rows_exclusive"], g["adaln_in_features"], g["adaln_out_features"]
-    for M in (1, 2, lim):
+    for M in (1, 2, 4):
         assert w8a8.select(M, N, K)["variant_name"] == "gemv"
-    assert w8a8.select(lim + 1, N, K)["variant_name"].startswith("gemm")
+    for M in (5, lim, lim + 1):
+        assert w8a8.select(M, N, K)["variant_name"].startswith("gemm")
+    assert w8a8.select(lim, N, K, variant=B.VARIANT_GEMV)["variant_name"] == "gemv"
     assert w8a8.workspace_size(1, N, K) == 0
+
+
+def test_selector_one_row_block_narrow_n_takes_64_column_tiles():
+    assert w8a8.select(17, 3072, 3072)["variant_name"] == "gemm_bn64"
+    assert w8a8.select(64, 9216, 3072)["variant_name"] == "gemm_bn128"   # 72 tiles already
+    p = w8a8.select(100, 3072, 12288)
+    assert p["variant_name"] == "gemm_bn64" and p["tile_n"] == 64 and p["num_tiles"] == 48
 
 
 def test_selector_gemm_plans():
@@ -115,7 +128,7 @@ def test_selector_gemm_plans():
     assert p["num_tiles"] == 17 * 12 and p["grid"] == 148
     # tiny output: few tiles, grid = tiles
     p = w8a8.select(64, 128, 256)
-    assert p["grid"] == p["num_tiles"] == 1
+    assert p["grid"] == p["num_tiles"] <= 2
     # GEMV would need more than 227 KB of shared memory: falls back to GEMM
     assert w8a8.select(16, 64, 16384)["variant_name"].startswith("gemm")
     # forced variants
@@ -237,7 +250,7 @@ def test_pair_k_split_plans():
 def test_selector_is_total_and_consistent(M, KN):
     K, N = KN
     p = w8a8.select(M, N, K)
-    assert p["variant_name"] in ("gemm_bn128", "gemm_bn256", "gemm_pair")
+    assert p["variant_name"] in ("gemm_bn64", "gemm_bn128", "gemm_bn256", "gemm_pair")
     tm, tn = p["tile_m"], p["tile_n"]
     assert p["num_tiles"] == -(-M // tm) * -(-N // tn)
     assert 1 <= p["grid"] <= 148

@@ -7,7 +7,8 @@ dequantization/bias epilogue producing bf16.  The kernels live in
 ``libw8a8.so`` (C ABI: ``include/w8a8.h``); this package is its binding.
 """
 from .binding import (  # noqa: F401
-    LIB_PATH, VARIANT_AUTO, VARIANT_GEMM_BN128, VARIANT_GEMM_BN256, VARIANT_GEMM_PAIR, VARIANT_GEMV,
+    LIB_PATH, VARIANT_AUTO, VARIANT_GEMM_BN64, VARIANT_GEMM_BN128, VARIANT_GEMM_BN256,
+    VARIANT_GEMM_PAIR, VARIANT_GEMV,
     W8A8Error, last_device_error, lib, linear, linear_fused, linear_fused_host, quant_act,
     quantize_weights, select, selftest_bounded_wait, status_string, unpack_int32_weights, version,
     workspace_size,

@@ -37,7 +37,9 @@ VARIANT_GEMV = 1
 VARIANT_GEMM_BN128 = 2
 VARIANT_GEMM_BN256 = 3
 VARIANT_GEMM_PAIR = 4
-VARIANT_NAMES = {0: "auto", 1: "gemv", 2: "gemm_bn128", 3: "gemm_bn256", 4: "gemm_pair"}
+VARIANT_GEMM_BN64 = 5
+VARIANT_NAMES = {0: "auto", 1: "gemv", 2: "gemm_bn128", 3: "gemm_bn256", 4: "gemm_pair",
+                 5: "gemm_bn64"}
 
 
 class W8A8Error(RuntimeError):

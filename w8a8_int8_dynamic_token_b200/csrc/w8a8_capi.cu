@@ -24,6 +24,7 @@ constexpr int64_t kMaxK = 133144;  // 127 * 127 * K <= 2^31 - 1
 constexpr int kMaxDevices = 64;
 constexpr int kGemmStages256 = 4;  // 4 x 48 KB ring for 128x256 tiles
 constexpr int kGemmStages128 = 6;  // 6 x 32 KB ring for 128x128 tiles
+constexpr int kGemmStages64 = 8;   // 8 x 24 KB ring for 128x64 tiles
 constexpr int kGemmStagesPair = 6; // 6 x 32 KB ring per CTA for 256x256 pair tiles
 constexpr int kGemmGroupM = 8;
 // K-split tail of the pair kernel (in 128-deep k-blocks): shortest piece a
@@ -102,13 +103,24 @@ inline bool gemv_fits(int64_t M, int64_t K, int max_smem) {
   return M <= kGemvMaxM && M * K + 1024 <= static_cast<int64_t>(max_smem);
 }
 
+// The selector takes the GEMV up to this many rows.  Measured on a B200 (the
+// whole layer, CUDA graphs): the GEMV streams the weight at 4-5 TB/s at M = 1
+// and its per-row dot products cost about 1.8 us per extra row at N = 9216,
+// K = 3072, while the tcgen05 GEMM path costs 12-16 us flat for M <= 128
+// there (launch, pipeline fill and epilogue bound); they cross at M = 5-6.
+constexpr int64_t kGemvAutoMaxM = 4;
+
 int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int max_smem,
                 w8a8_plan *plan) {
   if (sms < 1) return W8A8_ERR_INVALID_ARG;
   int v = variant;
   if (v == W8A8_VARIANT_AUTO) {
-    if (gemv_fits(M, K, max_smem)) {
+    if (M <= kGemvAutoMaxM && gemv_fits(M, K, max_smem)) {
       v = W8A8_VARIANT_GEMV;
+    } else if (M <= kBM && cdiv(N, 128) * 3 <= sms) {
+      // one row block and few 128-column tiles: 64-column tiles put twice as
+      // many CTAs on the weight stream (measured ~4% faster at N = 3072)
+      v = W8A8_VARIANT_GEMM_BN64;
     } else {
       // wave efficiency of each tile width; 256-wide tiles move half the
       // activation bytes per op, so 128-wide tiles must win clearly
@@ -197,8 +209,9 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     }
     return W8A8_OK;
   }
-  if (v != W8A8_VARIANT_GEMM_BN128 && v != W8A8_VARIANT_GEMM_BN256) return W8A8_ERR_INVALID_ARG;
-  const int bn = v == W8A8_VARIANT_GEMM_BN128 ? 128 : 256;
+  if (v != W8A8_VARIANT_GEMM_BN64 && v != W8A8_VARIANT_GEMM_BN128 && v != W8A8_VARIANT_GEMM_BN256)
+    return W8A8_ERR_INVALID_ARG;
+  const int bn = v == W8A8_VARIANT_GEMM_BN64 ? 64 : (v == W8A8_VARIANT_GEMM_BN128 ? 128 : 256);
   const int64_t tiles = cdiv(M, kBM) * cdiv(N, bn);
   if (tiles > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
   plan->tile_m = kBM;
@@ -630,6 +643,12 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
                : launch_gemm_pair<false, false>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc,
                                                 split, nullptr, stream);
   }
+  if (plan.variant == W8A8_VARIANT_GEMM_BN64) {
+    return acc ? launch_gemm_t<64, kGemmStages64, true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y,
+                                                         ldy, acc, stream)
+               : launch_gemm_t<64, kGemmStages64, false>(plan, q, s_a, M, K, Wq, s_w, bias, N,
+                                                          y, ldy, acc, stream);
+  }
   if (plan.variant == W8A8_VARIANT_GEMM_BN128) {
     return acc ? launch_gemm_t<128, kGemmStages128, true>(plan, q, s_a, M, K, Wq, s_w, bias, N,
                                                            y, ldy, acc, stream)
@@ -789,7 +808,7 @@ int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K, cons
                    const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
                    int32_t *acc_debug, int variant, void *workspace, size_t ws_bytes,
                    w8a8_stream_t stream) {
-  if (variant < W8A8_VARIANT_AUTO || variant > W8A8_VARIANT_GEMM_PAIR)
+  if (variant < W8A8_VARIANT_AUTO || variant > W8A8_VARIANT_GEMM_BN64)
     return W8A8_ERR_INVALID_ARG;
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant, workspace,
                      ws_bytes, reinterpret_cast<cudaStream_t>(stream));
