@@ -47,6 +47,20 @@ struct GemvParams {
   float *s_a_out;     // fused variant: optional copy of s_a
 };
 
+// Block-wide max of bit patterns of non-negative floats.
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();  // red[] may still be read from the previous call
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = 0u;
+#pragma unroll
+  for (int w = 0; w < kGemvThreads / 32; ++w) v = max(v, red[w]);
+  return v;
+}
+
 constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kGemvRows = 2;  // weight rows per warp step
 constexpr int kGemvVec = 8;   // 16-byte weight vectors per lane per row per step
@@ -73,6 +87,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_i8_kernel(const GemvParams 
   extern __shared__ __align__(16) uint8_t gemv_smem[];
   int8_t *qs = reinterpret_cast<int8_t *>(gemv_smem);  // [M][K]
   __shared__ float sas[kGemvMaxM];
+  __shared__ uint32_t red[kGemvWarps];
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -90,9 +105,25 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_i8_kernel(const GemvParams 
   if (pi < npairs) gemv_load(p.wq, p.N, nvec16, pi * kGemvRows, 0, lane, wv);
   grid_dependency_wait();
 
-  // ---- 1. activation rows -> shared memory (int8) + scales; in the fused
-  // variant one warp per row, up to 8 rows at once (no block-wide barriers)
-  if constexpr (FUSED) {
+  // ---- 1. activation rows -> shared memory (int8) + scales.  Fused, up to
+  // 4 rows: the whole block works on one row at a time (shortest latency
+  // per row); more rows: one warp per row, 8 rows at once.
+  if constexpr (FUSED && MT <= 4) {
+    const int nvec8 = K >> 3;
+    for (int m = 0; m < p.M; ++m) {
+      const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(m) * p.ldx);
+      float mm = 0.0f;
+      for (int v = tid; v < nvec8; v += kGemvThreads) mm = absmax_vec8(__ldg(xr + v), mm);
+      const float amax = __uint_as_float(block_max_u32(__float_as_uint(mm), red));
+      const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+      const bool fast = quant_fast_ok(sc);
+      const float rc = fast ? __frcp_rn(sc) : 0.0f;
+      if (tid == 0) sas[m] = sc;
+      uint2 *qrow = reinterpret_cast<uint2 *>(qs + m * K);
+      for (int v = tid; v < nvec8; v += kGemvThreads)
+        qrow[v] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(__ldg(xr + v), sc, rc, fast);
+    }
+  } else if constexpr (FUSED) {
     for (int m = warp; m < p.M; m += kGemvWarps)
       quant_row_by_warp<12>(p.x + static_cast<int64_t>(m) * p.ldx, K, qs + m * K, &sas[m], lane);
   } else {
