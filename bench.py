@@ -286,11 +286,22 @@ def timed(fn, steps: int, warmup: int, dist=None, sampler=None, graph=False):
     if dist is not None:
         dist.barrier()
     t = e0.elapsed_time(e1) / 1e3
-    if dist is not None:
-        tt = torch.tensor([t], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
-    return t
+    return max_over_ranks(t, dist)
+
+
+def max_over_ranks(seconds: float, dist=None, device="cuda") -> float:
+    """The slowest rank's time (every rank gets it): the job's time."""
+    if dist is None:
+        return seconds
+    tt = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_rate(units_per_step_per_rank: float, steps: int, seconds: float, world: int) -> float:
+    """Whole-job throughput of `world` replicas: the units all ranks processed
+    over the (max-over-ranks) time."""
+    return world * units_per_step_per_rank * steps / seconds
 
 
 class _Null:
@@ -376,7 +387,7 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device error after the timed region: {w8a8.status_string(status)}")
     sec_per_step = t / args.steps
-    value = world * ops * args.steps / t / 1e12
+    value = job_rate(ops, args.steps, t, world) / 1e12
 
     # the same layer with the host launch cost removed (CUDA graph of the steps)
     layer.i = 0
@@ -436,7 +447,7 @@ def run_ours(args):
     if not args.no_e2e:
         esteps = max(3, min(args.steps, 20))
         te, h2d, d2h = e2e_measure(layer, esteps, 2, dist)
-        e2e = {"value": round(world * ops * esteps / te / 1e12, 3), "unit": "TOPS",
+        e2e = {"value": round(job_rate(ops, esteps, te, world) / 1e12, 3), "unit": "TOPS",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(te / esteps * 1e3, 3)}
     del layer
