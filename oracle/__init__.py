@@ -54,6 +54,8 @@ def _load():
     lib.w8a8_oracle_epilogue.restype = ctypes.c_int
     lib.w8a8_oracle_linear.argtypes = [vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp]
     lib.w8a8_oracle_linear.restype = i64
+    lib.w8a16_oracle_linear.argtypes = [vp, i64, i64, i64, vp, vp, vp, i64, vp, vp, vp, vp]
+    lib.w8a16_oracle_linear.restype = ctypes.c_int
     lib.w8a8_oracle_pack_int32.argtypes = [vp, i64, i64, vp]
     lib.w8a8_oracle_pack_int32.restype = None
     lib.w8a8_oracle_unpack_int32.argtypes = [vp, i64, i64, vp]
@@ -180,6 +182,28 @@ def linear(x_bits: np.ndarray, wq: np.ndarray, s_w: np.ndarray, bias_bits=None) 
     if ov > 0:
         raise OverflowError(f"{ov} accumulators do not fit int32")
     return {"q": q, "s_a": s_a, "acc": acc, "y32": y32, "y": y}
+
+
+def w8a16_linear(x_bits: np.ndarray, wq: np.ndarray, s_w: np.ndarray, bias_bits=None) -> dict:
+    """Weight-only int8 layer on bf16 activations: y = bf16(acc32 * s_w + bias)
+    with acc32 = the exact sum_k x * q rounded once to fp32.  Returns acc32,
+    abs_sum (sum_k |x * q|, for summation-order bounds), y32 and y (bf16 bits)."""
+    x_bits = _as_c(x_bits, np.uint16)
+    wq = _as_c(wq, np.int8)
+    s_w = _as_c(s_w, np.float32)
+    M, K = x_bits.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K or s_w.shape[0] != N:
+        raise ValueError("shape mismatch")
+    b = None if bias_bits is None else _as_c(bias_bits, np.uint16)
+    out = {k: np.empty((M, N), np.float32) for k in ("acc32", "abs_sum", "y32")}
+    out["y"] = np.empty((M, N), np.uint16)
+    st = _load().w8a16_oracle_linear(_ptr(x_bits), M, K, K, _ptr(wq), _ptr(s_w),
+                                     None if b is None else _ptr(b), N, _ptr(out["acc32"]),
+                                     _ptr(out["abs_sum"]), _ptr(out["y32"]), _ptr(out["y"]))
+    if st != 0:
+        raise ValueError("w8a16_oracle_linear: bad arguments")
+    return out
 
 
 def pack_int32(wq: np.ndarray) -> np.ndarray:

@@ -184,6 +184,56 @@ int64_t w8a8_oracle_linear(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
     return ov;
 }
 
+/* ---- W8A16: int8 weights, bf16 activations ------------------------------- */
+
+/*
+ * The weight-only variant the pages ran first ("Issue 5 probe: int8 quantized
+ * DiT serve paths on the RTX 3090 (24 GB)", section "Round one: int8
+ * weight-only via compressed-tensors": int8 weight-only (W8A16),
+ * per-output-channel symmetric; the activations stay bf16).  With one scale
+ * per output channel the dequantized product factors as
+ *     y[m][n] = s_w[n] * sum_k x[m][k] * q[n][k] + bias[n].
+ * Each product x * q is exact in binary32 (an 8-bit significand times a
+ * 7-bit integer), so the only rounding inside the sum is the summation
+ * itself, whose order a tensor core leaves open.  The oracle forms the sum in
+ * binary64 (exact whenever the products span fewer than about 53 - 15 -
+ * log2 K binades, as for the tests' inputs; in general within K * 2^-53 of
+ * the exact sum, relative to sum |x * q|), rounds it once to binary32
+ * (acc32), then applies the scale and the bias as separately rounded
+ * binary32 operations and rounds to bf16:
+ *     y32 = acc32 * s_w[n] (+ (float)bias[n]),  y = bf16(y32).
+ * abs_sum[m][n] = sum_k |x * q| (binary64, rounded to binary32) bounds how
+ * far any binary32 summation order can drift from the exact sum:
+ * |sum_fp32 - sum| <= gamma_K * abs_sum,  gamma_K = K u / (1 - K u),
+ * u = 2^-24 (the standard bound for recursive summation in any order).
+ */
+int w8a16_oracle_linear(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                        const int8_t *wq, const float *s_w, const uint16_t *bias, int64_t N,
+                        float *acc32_out, float *abs_sum_out, float *y32_out, uint16_t *y_out)
+{
+    if (!x || !wq || !s_w || M < 0 || N < 0 || K < 0 || ldx < K) return -1;
+    if (fegetround() != FE_TONEAREST) fesetround(FE_TONEAREST);
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double sum = 0.0, asum = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = (double)bf16_to_f32(x[m * ldx + k]) * (double)wq[n * K + k];
+                sum += p;
+                asum += fabs(p);
+            }
+            float acc = (float)sum;
+            float v = acc * s_w[n];
+            if (bias) v = v + bf16_to_f32(bias[n]);
+            if (acc32_out) acc32_out[m * N + n] = acc;
+            if (abs_sum_out) abs_sum_out[m * N + n] = (float)asum;
+            if (y32_out) y32_out[m * N + n] = v;
+            if (y_out) y_out[m * N + n] = f32_to_bf16_rne(v);
+        }
+    }
+    return 0;
+}
+
 /* ---- packed int32 weight storage ----------------------------------------- */
 
 /*

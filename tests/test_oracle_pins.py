@@ -435,3 +435,70 @@ def test_planted_packing_mistakes_fail_pin():
     good = oracle.pack_int32(wq)
     assert not np.array_equal(be, good) and not np.array_equal(raw, good)
     assert oracle.unpack_int32(be, 4).tolist() != wq.tolist()
+
+
+# --------------------------------------------------------------------------
+# W8A16 (int8 weight-only, bf16 activations): y = bf16(acc32 * s_w + bias),
+# acc32 = sum_k x * q rounded once to fp32 ("Issue 5 probe ...", section
+# "Round one: int8 weight-only via compressed-tensors": per-output-channel
+# symmetric int8 weights, activations kept bf16).
+# --------------------------------------------------------------------------
+
+def test_w8a16_worked_example():
+    x = bits([[1.0, 2.0, 0.5, -4.0]])
+    wq = np.array([[127, -1, 2, 3]], np.int8)
+    r = oracle.w8a16_linear(x, wq, np.array([0.5], np.float32), bits([0.25])[0])
+    # 127 - 2 + 1 - 12 = 114; 114 * 0.5 = 57; + 0.25 = 57.25 (exact in bf16)
+    assert r["acc32"][0, 0] == 114.0 and r["abs_sum"][0, 0] == 127 + 2 + 1 + 12
+    assert r["y32"][0, 0] == 57.25 and f64(r["y"])[0, 0] == 57.25
+
+
+def test_w8a16_sum_is_the_exact_sum_rounded_once():
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    x = synth.make_x(3, 96, "studentt", 11)
+    wq = rng.integers(-127, 128, size=(5, 96), dtype=np.int8)
+    r = oracle.w8a16_linear(x, wq, np.ones(5, np.float32))
+    xf = f64(x)
+    for m in range(3):
+        for n in range(5):
+            exact = sum(Fraction(float(xf[m, k])) * int(wq[n, k]) for k in range(96))
+            assert r["acc32"][m, n] == np.float32(float(exact))       # one rounding, to nearest
+            assert r["abs_sum"][m, n] == np.float32(float(sum(abs(Fraction(float(xf[m, k])) * int(wq[n, k])) for k in range(96))))
+
+
+def test_w8a16_matches_dequantized_matmul():
+    x = synth.make_x(8, 256, "studentt", 12)
+    w = synth.make_w(16, 256, 12)
+    wq, sw = oracle.quantize_weights(w)
+    b = synth.make_bias(16, 12)
+    r = oracle.w8a16_linear(x, wq, sw, b)
+    ref = f64(x) @ (wq.astype(np.float64) * sw[:, None].astype(np.float64)).T + f64(b)[None, :]
+    # acc32 rounding, then two fp32 operations: a few fp32 ulps of the terms involved
+    tol = (np.abs(r["acc32"]).astype(np.float64) * np.abs(sw)[None, :] + np.abs(f64(b))[None, :]) * 2.0 ** -22
+    assert np.all(np.abs(r["y32"] - ref) <= tol + 1e-30)
+
+
+def test_w8a16_on_integer_activations_equals_the_w8a8_accumulator():
+    # bf16 integers in [-127, 127] are their own int8 codes with s_a = 1, so the
+    # two oracle paths must produce the same accumulator and, with s_a = 1, y32
+    rng = np.random.default_rng(13)
+    q = rng.integers(-127, 128, size=(4, 64)).astype(np.float64)
+    x = bits(q)
+    wq = rng.integers(-127, 128, size=(6, 64), dtype=np.int8)
+    sw = (rng.random(6) * 0.01 + 1e-3).astype(np.float32)
+    r16 = oracle.w8a16_linear(x, wq, sw)
+    acc8 = oracle.gemm_i32(q.astype(np.int8), wq)
+    assert np.array_equal(r16["acc32"], acc8.astype(np.float32))
+    y32_8, _ = oracle.epilogue(acc8, np.ones(4, np.float32), sw, None)
+    assert np.array_equal(r16["y32"], y32_8)
+
+
+def test_planted_w8a16_mistakes_fail_pin():
+    x = bits([[1.0, 2.0, 0.5, -4.0]])
+    wq = np.array([[127, -1, 2, 3]], np.int8)
+    good = oracle.w8a16_linear(x, wq, np.array([0.5], np.float32))["y32"][0, 0]
+    assert good == 57.0
+    assert oracle.w8a16_linear(x, wq, np.array([1.0], np.float32))["y32"][0, 0] != 57.0   # scale dropped
+    assert oracle.w8a16_linear(x, -wq, np.array([0.5], np.float32))["y32"][0, 0] != 57.0  # sign
+    assert oracle.w8a16_linear(x, wq[:, ::-1].copy(), np.array([0.5], np.float32))["y32"][0, 0] != 57.0
