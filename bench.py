@@ -538,7 +538,37 @@ def extra_components(args, dev, dist, peaks, world):
         out["dit_block"] = dit_block_component(dev, dist, max(10, steps // 4))
         out["small_m"] = small_m_component(dev, dist, peaks, steps)
         out["unpack_int32_weights"] = unpack_component(dev, dist, peaks, steps)
+        out["w8a16_qkv"] = w8a16_component(dev, dist, peaks, steps)
     return out
+
+
+def w8a16_component(dev, dist, peaks, steps):
+    """The weight-only variant on the QKV shape: bf16 x [4352, 3072] against
+    int8 Wq [9216, 3072] widened to bf16 in the kernel, bf16 tensor cores."""
+    import w8a8_int8_dynamic_token_b200 as w8a8
+    case = synth.QKV
+    M, K, N = case.M, case.K, case.N
+    W = bf16_dev(case.w(), dev)
+    Wq, s_w = w8a8.quantize_weights(W)
+    del W
+    x0 = bf16_dev(case.x(), dev)
+    nsets = n_sets(2 * M * K + N * K + 2 * M * N)
+    sets = [(x0.clone(), Wq.clone(), torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+            for _ in range(nsets)]
+    i = [0]
+
+    def step():
+        x, wq, y = sets[i[0] % nsets]
+        i[0] += 1
+        w8a8.w8a16_linear(x, wq, s_w, out=y)
+
+    t = timed(step, steps, 5, dist, graph=True) / steps
+    tflops = case.ops / t / 1e12
+    del sets
+    torch.cuda.empty_cache()
+    return {"us": round(t * 1e6, 2), "TFLOPS": round(tflops, 1),
+            "frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
+            "peak_basis": "measured bf16 burst (MEASURED_PEAKS.json)"}
 
 
 def small_m_component(dev, dist, peaks, steps):

@@ -235,6 +235,22 @@ W8A8_API int w8a8_linear_fused_host(const void *x_host, int64_t M, int64_t K,
                            void *workspace, size_t ws_bytes, w8a8_stream_t stream);
 
 /*
+ * The weight-only variant (W8A16): int8 weights with per-output-channel fp32
+ * scales, bf16 activations used as they are ("Issue 5 probe: int8 quantized
+ * DiT serve paths on the RTX 3090 (24 GB)", section "Round one: int8
+ * weight-only via compressed-tensors").  x bf16 [M,K] (row stride ldx),
+ * Wq int8 [N,K] dense, s_w fp32 [N], bias bf16 [N] or NULL -> y bf16 [M,N]
+ * (row stride ldy):  y = bf16( (sum_k x[m,k] * Wq[n,k]) * s_w[n] + bias[n] ),
+ * the sum accumulated in fp32 by the tensor cores (order unspecified; each
+ * product is exact), the scale and bias applied once as rounded fp32
+ * operations.  The int8 weights are widened to bf16 inside the kernel; no
+ * workspace.  Preconditions as for w8a8_linear_fused.
+ */
+W8A8_API int w8a16_linear(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
+                          const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null,
+                          int64_t N, void *y_bf16, int64_t ldy, w8a8_stream_t stream);
+
+/*
  * Host-only: the selector's plan for (M, N, K) on a device with num_sms SMs
  * (148 on B200).  Pure function of its arguments; needs no GPU.
  */

@@ -21,7 +21,7 @@ import synth
 import w8a8_int8_dynamic_token_b200 as w8a8
 from w8a8_int8_dynamic_token_b200 import binding as B
 
-from gpu_util import bf16_to_f64, bits_of, check_y, f32_bits, sample_rows, to_dev
+from gpu_util import bf16_to_f64, bf16_ulp, bits_of, check_y, f32_bits, sample_rows, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -607,3 +607,38 @@ def test_quantization_fused_into_pair_launch(M, N, K, ldx):
     rows = sample_rows(M, seed=17, n_random=32)
     y32, y_ref = oracle.epilogue(oracle.gemm_i32(q_ref[rows], wq), s_ref[rows], sw, b)
     assert check_y(bits_of(y1)[rows], y_ref, y32, "fused launch") == 0
+
+
+# ----------------------------------------------------------------- W8A16 (weight-only)
+
+W8A16_CASES = [(64, 128, 256, True), (300, 520, 400, True), (129, 1032, 3072, False),
+               (17, 264, 12288, True), (4352, 9216, 3072, True)]
+
+
+@pytest.mark.parametrize("M,N,K,bias", W8A16_CASES)
+def test_w8a16_vs_oracle(M, N, K, bias):
+    """y = bf16((x @ Wq^T) * s_w + bias) with fp32 tensor-core accumulation in
+    an unspecified order: each output must lie within one bf16 ulp of the
+    oracle's fp32 value plus the bound on any fp32 summation order,
+    |s_w| * gamma_K * sum_k |x q| (gamma_K = K u / (1 - K u), u = 2^-24), plus
+    the two fp32 roundings of the epilogue."""
+    x = synth.make_x(M, K, "studentt", 21)
+    w = synth.make_w(N, K, 21)
+    wq, sw = oracle.quantize_weights(w)
+    b = synth.make_bias(N, 21) if bias else None
+    y = w8a8.w8a16_linear(to_dev(x), torch.from_numpy(wq).cuda(), torch.from_numpy(sw).cuda(),
+                          to_dev(b) if b is not None else None)
+    torch.cuda.synchronize()
+    rows = np.arange(M) if M <= 512 else sample_rows(M, seed=21, n_random=32)
+    r = oracle.w8a16_linear(np.ascontiguousarray(x[rows]), wq, sw, b)
+    got = bf16_to_f64(bits_of(y)[rows])
+    ref = r["y32"].astype(np.float64)
+    u = 2.0 ** -24
+    gamma = K * u / (1 - K * u)
+    tol = (bf16_ulp(ref) + np.abs(sw.astype(np.float64))[None, :] * gamma * r["abs_sum"]
+           + 4 * u * np.abs(ref) + 1e-30)
+    assert np.isfinite(got).all()
+    bad = np.abs(got - ref) > tol
+    assert not bad.any(), f"{int(bad.sum())} outputs outside the bound, first {np.argwhere(bad)[:3].tolist()}"
+    # most outputs round to the oracle's bf16 value exactly
+    assert np.mean(bits_of(y)[rows] == r["y"]) > 0.9

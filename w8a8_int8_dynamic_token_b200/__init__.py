@@ -11,5 +11,5 @@ from .binding import (  # noqa: F401
     VARIANT_GEMM_PAIR, VARIANT_GEMV,
     W8A8Error, last_device_error, lib, linear, linear_fused, linear_fused_host, quant_act,
     quantize_weights, select, selftest_bounded_wait, status_string, unpack_int32_weights, version,
-    workspace_size,
+    w8a16_linear, workspace_size,
 )

@@ -82,6 +82,7 @@ _SIGNATURES = {
                                 _vp], _int),
     "w8a8_linear_fused_noalloc": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp],
                                   _int),
+    "w8a16_linear": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp], _int),
     "w8a8_select": ([_i64, _i64, _i64, _i32, _int, ctypes.POINTER(Plan)], _int),
     "w8a8_last_device_error": ([_vp], _int),
     "w8a8_selftest_bounded_wait": ([_i64, _vp], _int),
@@ -93,7 +94,7 @@ def header_functions() -> list[str]:
     """Names of the functions include/w8a8.h declares."""
     with open(HEADER_PATH) as f:
         text = f.read()
-    return sorted(set(re.findall(r"W8A8_API\s+[^;(]*?\b(w8a8_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"W8A8_API\s+[^;(]*?\b(w8a(?:8|16)_\w+)\s*\(", text)))
 
 
 def lib() -> ctypes.CDLL:
@@ -181,6 +182,10 @@ def w8a8_linear_fused_host(x_host, M, K, Wq, s_w, bias, N, y_host, x_dev, y_dev,
 
 def w8a8_linear_fused_noalloc(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, stream) -> int:
     return lib().w8a8_linear_fused_noalloc(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, stream)
+
+
+def w8a16_linear_raw(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, stream) -> int:
+    return lib().w8a16_linear(x, M, K, ldx, Wq, s_w, bias, N, y, ldy, stream)
 
 
 def w8a8_select(M, N, K, num_sms=148, variant=VARIANT_AUTO) -> tuple[int, Plan]:
@@ -351,6 +356,26 @@ def linear_fused(x, Wq, s_w, bias=None, out=None, workspace=None, return_interme
                              _stream(stream)), "w8a8_linear_fused")
     if return_intermediates:
         return y, q, s_a
+    return y
+
+
+def w8a16_linear(x, Wq, s_w, bias=None, out=None, stream=None):
+    """Weight-only int8 layer on bf16 x [M, K]: y = bf16((x @ Wq^T) * s_w + bias),
+    fp32 accumulation on the tensor cores."""
+    _need(x, "x", torch.bfloat16, 2)
+    dev = x.device
+    _need(Wq, "Wq", torch.int8, 2, dev)
+    _need(s_w, "s_w", torch.float32, 1, dev)
+    M, K = x.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] != K or s_w.shape[0] != N or not Wq.is_contiguous():
+        raise ValueError("shape mismatch between x, Wq, s_w")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1, dev)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(y, "out", torch.bfloat16, 2, dev)
+    _check(w8a16_linear_raw(_ptr(x), M, K, x.stride(0), _ptr(Wq), _ptr(s_w), _ptr(bias), N,
+                            _ptr(y), y.stride(0), _stream(stream)), "w8a16_linear")
     return y
 
 

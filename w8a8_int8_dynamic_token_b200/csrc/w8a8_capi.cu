@@ -15,6 +15,7 @@
 #include "w8a8_gemm.cuh"
 #include "w8a8_gemv.cuh"
 #include "w8a8_pack.cuh"
+#include "w8a16_gemm.cuh"
 #include "w8a8_ptx.cuh"
 #include "w8a8_quant.cuh"
 
@@ -301,6 +302,38 @@ int encode_i8_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, i
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+}
+
+// bf16 matrix [rows, cols] with row stride ld elements, box 64 (cols) x
+// box_rows, 128-byte swizzle (the W8A16 GEMM's activation operand).
+int encode_bf16_load_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols,
+                         int64_t ld, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return W8A8_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kW16BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+}
+
+// int8 matrix [rows, K] dense, box 64 (K) x box_rows, no swizzle (the W8A16
+// GEMM's weights, widened to bf16 in shared memory by the kernel).
+int encode_i8_plain_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K,
+                        int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
+  if (enc == nullptr) return W8A8_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kW16BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
 }
@@ -955,6 +988,57 @@ int w8a8_linear_fused_host(const void *x_host, int64_t M, int64_t K, const int8_
     return W8A8_ERR_CUDA;
   }
   return W8A8_OK;
+}
+
+int w8a16_linear(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t *Wq,
+                 const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
+                 w8a8_stream_t stream) {
+  if (!x || !Wq || !s_w || !y) return W8A8_ERR_INVALID_ARG;
+  int st = check_mk(M, K, ldx);
+  if (st != W8A8_OK) return st;
+  st = check_n(N, ldy);
+  if (st != W8A8_OK) return st;
+  if (!aligned16(x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(y) ||
+      (bias && !aligned16(bias)))
+    return W8A8_ERR_MISALIGNED;
+  const DeviceInfo *d = nullptr;
+  st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  constexpr int BN = 128, STAGES = 4;
+  using L = W16Layout<BN, STAGES>;
+  CUtensorMap mx, mw, my;
+  st = encode_bf16_load_map(&mx, x, M, K, ldx, kBM);
+  if (st != W8A8_OK) return st;
+  st = encode_i8_plain_map(&mw, Wq, N, K, BN);
+  if (st != W8A8_OK) return st;
+  st = encode_bf16_store_map(&my, y, M, N, ldy);
+  if (st != W8A8_OK) return st;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = static_cast<int32_t>(M);
+  p.N = static_cast<int32_t>(N);
+  p.K = static_cast<int32_t>(K);
+  p.num_m_blk = static_cast<int32_t>(cdiv(M, kBM));
+  p.num_n_blk = static_cast<int32_t>(cdiv(N, BN));
+  const int64_t tiles = static_cast<int64_t>(p.num_m_blk) * p.num_n_blk;
+  if (tiles > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  p.num_tiles = static_cast<int32_t>(tiles);
+  p.k_blocks = static_cast<int32_t>(cdiv(K, kW16BK));
+  p.group_m = kGemmGroupM;
+  p.s_a = nullptr;
+  p.s_w = s_w;
+  p.bias = static_cast<const uint16_t *>(bias);
+  p.y = static_cast<uint16_t *>(y);
+  p.ldy = ldy;
+  p.acc_out = nullptr;
+  p.dp_tiles = p.num_tiles;
+  p.tail_nsplit = 1;
+  constexpr auto kernel = gemm_w8a16_tcgen05_kernel<BN, STAGES>;
+  st = ensure_smem_limit<kernel>(L::kSmemBytes);
+  if (st != W8A8_OK) return st;
+  const int64_t grid = tiles < d->sms ? tiles : d->sms;
+  return launch_ex(true, kernel, dim3(static_cast<unsigned>(grid)), dim3(kW16Threads),
+                   L::kSmemBytes, reinterpret_cast<cudaStream_t>(stream), mx, mw, my, p);
 }
 
 int w8a8_last_device_error(w8a8_stream_t stream) {
