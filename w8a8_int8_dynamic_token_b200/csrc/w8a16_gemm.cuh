@@ -53,6 +53,29 @@ struct W16Layout {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
+// Two int8 lanes of a word -> a bf16x2 word, exactly and with full-rate
+// integer/float operations only: sign-extend the byte (a byte permute with
+// the sign-replicate selector), add it to the bit pattern of 1.5 * 2^23 --
+// giving the float 1.5 * 2^23 + v exactly -- subtract 1.5 * 2^23 (exact,
+// = (float)v), and keep the upper halves: (float)v has at most 8 significant
+// bits, so its low 16 bits are zero and its upper half is bf16(v).
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t widen2(uint32_t w, uint32_t sel_lo, uint32_t sel_hi) {
+  const float magic = 12582912.0f;  // 1.5 * 2^23
+  // selector 0xNNNn, N = 8 + n: result byte 0 = byte n of w, bytes 1..3 =
+  // that byte's sign (prmt's sign-replicate selectors)
+  const uint32_t e0 = prmt_b32(w, 0u, sel_lo);
+  const uint32_t e1 = prmt_b32(w, 0u, sel_hi);
+  const float f0 = __fsub_rn(__uint_as_float(__float_as_uint(magic) + e0), magic);
+  const float f1 = __fsub_rn(__uint_as_float(__float_as_uint(magic) + e1), magic);
+  return prmt_b32(__float_as_uint(f0), __float_as_uint(f1), 0x7632u);
+}
+
 // int8 weights of one stage -> bf16 in the 128-byte-swizzled K-major layout:
 // row r (128 bytes = 64 bf16) holds its 16-byte chunk j at position j ^ (r & 7).
 // Thread `t` of the converter warps takes rows t, t + 128, ...
@@ -67,14 +90,8 @@ __device__ __forceinline__ void widen_stage(const uint8_t *b8, uint8_t *b16, int
       uint32_t o[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int32_t b0 = static_cast<int8_t>(w[i] & 0xFFu);
-        const int32_t b1 = static_cast<int8_t>((w[i] >> 8) & 0xFFu);
-        const int32_t b2 = static_cast<int8_t>((w[i] >> 16) & 0xFFu);
-        const int32_t b3 = static_cast<int8_t>(w[i] >> 24);
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(static_cast<float>(b0), static_cast<float>(b1));
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(static_cast<float>(b2), static_cast<float>(b3));
-        o[2 * i] = *reinterpret_cast<const uint32_t *>(&lo);
-        o[2 * i + 1] = *reinterpret_cast<const uint32_t *>(&hi);
+        o[2 * i] = widen2(w[i], 0x8880u, 0x9991u);
+        o[2 * i + 1] = widen2(w[i], 0xAAA2u, 0xBBB3u);
       }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
