@@ -353,9 +353,36 @@ def cpu_baseline(case: synth.LayerCase, budget_s: float = 12.0, max_rows: int = 
     oracle.linear(x[:rows], wq, sw, b)
     dt = time.perf_counter() - t0
     return {"value": 2.0 * rows * N * K / dt / 1e12, "unit": "TOPS", "cores": oracle.threads(),
+            "nproc": os.cpu_count(), "cpu_model": cpu_model(),
             "kind": "oracle", "seconds": round(dt, 3),
             "sample": f"first {rows} of {M} rows of the {case.name} layer (all {N} outputs per row): "
                       f"per-token quant + exact int32 GEMM + fp32 epilogue, plain C with OpenMP"}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def single_launch_us(fn, reps: int = 20) -> float:
+    """Median time of one isolated call: synchronize, then events around the
+    call alone (the device idle before it)."""
+    times = []
+    for _ in range(reps):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    return statistics.median(times)
 
 
 def run_ours(args):
@@ -431,8 +458,11 @@ def run_ours(args):
             roofline["frac_of_clock_peak"] = round(achieved / clock_peak, 4)
             roofline["clock_peak_tops"] = round(clock_peak, 1)
     quant_bytes = 3 * M * K + 4 * M
+    layer.i = 0
+    t_single = single_launch_us(layer.step)
     extras = {
         "layer_us": round(sec_per_step * 1e6, 2),
+        "layer_single_call_us": round(t_single, 2),
         "layer_us_graph": round(t_graph * 1e6, 2),
         "layer_tops_graph": round(ops / t_graph / 1e12, 1),
         "layer_frac_of_nominal_4500": round(ops / sec_per_step / 1e12 / NOMINAL_INT8_TOPS, 4),
@@ -473,6 +503,7 @@ def run_ours(args):
             "impl": "ours",
             "config": {"workload": f"{case.name}: x bf16 [{M},{K}] ({case.x_kind}) @ Wq int8 [{N},{K}] + bias -> y bf16",
                        "M": M, "K": K, "N": N, "seed": case.seed,
+                       "gpu": torch.cuda.get_device_name(dev),
                        "parallelism": f"replicas x{world}",
                        "l2": f"inputs rotate over independent buffer sets totalling > 2x the 126 MB L2",
                        "kernel_variant": layer_variant_name(case)},
