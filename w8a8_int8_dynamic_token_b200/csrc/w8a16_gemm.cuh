@@ -31,6 +31,97 @@
 
 namespace w8a8 {
 
+// D (fp32, TMEM) (+)= A (bf16, smem) x B (bf16, smem)^T, one CTA, K = 16.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor, kind::f16: D f32 (bits 4-5 = 1), A and B bf16
+// (bits 7-9 = 1, 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at
+// bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// One epilogue warp's share of an fp32 accumulator (its 32 TMEM lanes, COLS
+// columns from col_base, in 32-column chunks): y = bf16(acc * s_w + bias), the
+// multiply and the add separately rounded fp32 operations, stored through the
+// same 64-byte-swizzled staging buffers and TMA stores as the int8 GEMM's
+// epilogue.
+template <int COLS>
+__device__ __forceinline__ void w16_epilogue_warp_slice(const GemmParams &p,
+                                                        const CUtensorMap *tmap_y, uint32_t t_row,
+                                                        int row0, int col_base,
+                                                        uint8_t *stage_buf,
+                                                        uint32_t &chunk_count, int lane) {
+  if (row0 >= p.M) return;  // all 32 rows past M: nothing to store
+#pragma unroll 1
+  for (int c = 0; c < COLS; c += kEpiChunk) {
+    const int col0 = col_base + c;
+    if (col0 >= p.N) break;  // warp-uniform
+    float sw[32];
+    uint32_t bw[16];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const int cg = col0 + 8 * g;
+      if (cg < p.N) {
+        const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg));
+        const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.s_w + cg) + 1);
+        sw[8 * g + 0] = w0.x; sw[8 * g + 1] = w0.y; sw[8 * g + 2] = w0.z; sw[8 * g + 3] = w0.w;
+        sw[8 * g + 4] = w1.x; sw[8 * g + 5] = w1.y; sw[8 * g + 6] = w1.z; sw[8 * g + 7] = w1.w;
+        if (p.bias != nullptr) {
+          const uint4 braw = __ldg(reinterpret_cast<const uint4 *>(p.bias + cg));
+          bw[4 * g + 0] = braw.x; bw[4 * g + 1] = braw.y;
+          bw[4 * g + 2] = braw.z; bw[4 * g + 3] = braw.w;
+        } else {
+          bw[4 * g + 0] = bw[4 * g + 1] = bw[4 * g + 2] = bw[4 * g + 3] = 0u;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sw[8 * g + i] = 0.0f;
+        bw[4 * g + 0] = bw[4 * g + 1] = bw[4 * g + 2] = bw[4 * g + 3] = 0u;
+      }
+    }
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(t_row + c, r);
+    tmem_ld_wait();
+    uint32_t packed[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float2 v = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+      v = mul2_rn(v, make_float2(sw[2 * i], sw[2 * i + 1]));
+      if (p.bias != nullptr)
+        v = add2_rn(v, make_float2(__uint_as_float(bw[i] << 16),
+                                   __uint_as_float(bw[i] & 0xFFFF0000u)));
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+      packed[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    uint8_t *buf = stage_buf + (chunk_count & 1u) * kEpiBufBytes;
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int pos = j ^ ((lane >> 1) & 3);
+      *reinterpret_cast<uint4 *>(buf + lane * 64 + pos * 16) =
+          make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmap_y, buf, col0, row0);
+      bulk_commit_group();
+    }
+    ++chunk_count;
+  }
+}
+
 constexpr int kW16ConvWarps = 4;
 constexpr int kW16Threads = (2 + kEpiWarps + kW16ConvWarps) * 32;  // 448
 constexpr int kW16BK = 64;  // bf16 elements of K per stage = one 128-byte swizzle row
@@ -254,9 +345,8 @@ __global__ void __launch_bounds__(kW16Threads, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN + half * (BN / 2));
-      epilogue_warp_slice<BN / 2, false, true>(p, &tmap_y, t_row, mb * kBM + quarter * 32,
-                                               nb * BN + half * (BN / 2), stage_buf,
-                                               chunk_count, lane);
+      w16_epilogue_warp_slice<BN / 2>(p, &tmap_y, t_row, mb * kBM + quarter * 32,
+                                      nb * BN + half * (BN / 2), stage_buf, chunk_count, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);

@@ -263,9 +263,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) 
 // proper.
 constexpr int kEpiNormal = 0, kEpiWritePartial = 1, kEpiAddPartials = 2;
 
-// ACC_F32: the accumulators are fp32 (a bf16 x bf16 MMA) and there is no
-// activation scale: y = bf16(acc * s_w + bias).
-template <int COLS, bool RAW_OUT, bool ACC_F32 = false>
+template <int COLS, bool RAW_OUT>
 __device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const CUtensorMap *tmap_y,
                                                     uint32_t t_row, int row0, int col_base,
                                                     uint8_t *stage_buf, uint32_t &chunk_count,
@@ -277,7 +275,7 @@ __device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const C
   const bool row_ok = row < p.M;
   // s_a may have been written earlier in this same launch (fused
   // quantization): read it through L2, never the non-coherent path
-  const float sa = (row_ok && !ACC_F32) ? __ldcg(p.s_a + row) : 0.0f;
+  const float sa = row_ok ? __ldcg(p.s_a + row) : 0.0f;
   // a warp whose 32 rows all lie past M has nothing to store; a narrow tile
   // (ncols < COLS, a multiple of 32) has fewer chunks
   const int cols_here = row0 < p.M ? (ncols < COLS ? ncols : COLS) : 0;
@@ -369,14 +367,9 @@ __device__ __forceinline__ void epilogue_warp_slice(const GemmParams &p, const C
       const float2 sa2 = make_float2(sa, sa);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        float2 v;
-        if constexpr (ACC_F32) {
-          v = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-        } else {
-          v = make_float2(__int2float_rn(static_cast<int32_t>(r[2 * i])),
-                          __int2float_rn(static_cast<int32_t>(r[2 * i + 1])));
-          v = mul2_rn(v, sa2);
-        }
+        float2 v = make_float2(__int2float_rn(static_cast<int32_t>(r[2 * i])),
+                               __int2float_rn(static_cast<int32_t>(r[2 * i + 1])));
+        v = mul2_rn(v, sa2);
         v = mul2_rn(v, make_float2(sw[2 * i], sw[2 * i + 1]));
         if (p.bias != nullptr)
           v = add2_rn(v, make_float2(__uint_as_float(bw[i] << 16),
