@@ -265,3 +265,43 @@ def test_quantization_inside_the_gemm_launch_plan():
     assert w8a8.select(4352, 3072, 12288)["quant_in_gemm_launch"] == 0   # K > 3072
     assert w8a8.select(8704, 3072, 3072)["quant_in_gemm_launch"] == 0    # 8 passes
     assert w8a8.select(100, 3072, 3072)["quant_in_gemm_launch"] == 0     # not the pair kernel
+
+
+# Property check of the selector over random shapes (host only): every plan
+# covers the output exactly once with tiles the launch can hold.
+from hypothesis import given, settings, strategies as hst  # noqa: E402
+
+
+def _cdiv(a, b):
+    return -(-a // b)
+
+
+@settings(max_examples=400, deadline=None)
+@given(M=hst.integers(1, 20000), n8=hst.integers(1, 4000), k16=hst.integers(1, 2000))
+def test_selector_plans_are_valid_for_random_shapes(M, n8, k16):
+    N, K = 8 * n8, 16 * k16
+    p = w8a8.select(M, N, K)
+    v = p["variant_name"]
+    assert p["grid"] >= 1
+    if v == "gemv":
+        assert M <= 4 and M * K + 1024 <= 232448
+        return
+    tm, tn, tiles = p["tile_m"], p["tile_n"], p["num_tiles"]
+    assert tiles == _cdiv(M, tm) * _cdiv(N, tn)
+    assert p["grid"] <= 148
+    if v != "gemm_pair":
+        assert p["grid"] == min(tiles, 148)
+        assert not (p["split_tiles"] or p["tail_tiles_nsplit"])
+        return
+    assert tm == tn == 256 and p["grid"] % 2 == 0
+    pairs, kb = p["grid"] // 2, _cdiv(K, 128)
+    ns, st, per = p["tail_tiles_nsplit"], p["split_tiles"], p["split_kblocks_per_pair"]
+    assert not (ns and st)
+    if ns:
+        rem = tiles % pairs
+        assert tiles >= pairs and 0 < rem and 2 * rem <= pairs and ns == 2
+    if st:
+        assert per >= 24 and per * pairs >= st * kb and st < 2 * pairs
+        assert (tiles - st) % pairs == 0
+    if p["quant_in_gemm_launch"]:
+        assert K <= 3072 and _cdiv(M, p["grid"] * 8) <= 4
