@@ -299,7 +299,7 @@ W8A8_API int w8a8_selftest_bounded_wait(int64_t limit_ns, w8a8_stream_t stream);
  * execution overlaps on the GPU (different streams, or threads that do not
  * order their calls) race on the array -- the caller must serialize them.
  *
- * The paper has no counterpart to this entry point.
+ * The source pages describe no counterpart to this entry point.
  */
 W8A8_API int w8a8_linear_fused_noalloc(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
                                        const int8_t *Wq, const float *s_w,
