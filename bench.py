@@ -2,7 +2,8 @@
 """Benchmark of the W8A8 int8-dynamic linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload qkv|ffn_up|ffn_down] [--no-extras] [--no-cpu-baseline]
+                    [--workload qkv|ffn_up|ffn_down|adaln_m1|adaln_m2]
+                    [--no-extras] [--no-e2e] [--no-cpu-baseline] [--cpu-budget S]
 
 A step is one whole layer call on one batch: per-token quantization of the
 bf16 activations, the int8 tensor-core GEMM and the fused dequantization
@@ -16,6 +17,13 @@ synchronize on both sides, timed with CUDA events on the launching stream;
 the reported time is the max over ranks.  Between steps the inputs rotate
 over several independent buffer sets whose combined size exceeds twice the
 126 MB L2, so no step reads data a previous step left in L2.
+
+Beside the headline line's own figures (roofline of the dominant kernel,
+end-to-end time from pinned host buffers, CPU oracle baseline, clocks sampled
+during the timed region), `components` reports the other workloads: the
+AdaLN GEMV at M = 1 and 2, the FFN layers alone and back to back, one DiT
+block's linears at CFG batch 2, the small-M regime, packed-weight loading
+and the W8A16 variant.
 
 Multi-GPU: the layer shards into independent problems, so N ranks run N
 replicas with no collective on the data path (weak scaling); `value` is the
