@@ -580,9 +580,7 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
 }
 
 template <bool FUSED, bool RAW>
-int launch_gemv_m(const w8a8_plan &plan, const GemvParams &p, int max_smem, int sms,
-                  cudaStream_t stream) {
-  (void)sms;
+int launch_gemv_m(const w8a8_plan &plan, const GemvParams &p, cudaStream_t stream) {
   const int smem = p.M * p.K;
 #define W8A8_GEMV_CASE(MT)                                                              \
   {                                                                                     \
@@ -666,8 +664,8 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
     p.y = static_cast<uint16_t *>(y);
     p.ldy = ldy;
     p.acc_out = acc;
-    return acc ? launch_gemv_m<false, true>(plan, p, d->max_smem_optin, d->sms, stream)
-               : launch_gemv_m<false, false>(plan, p, d->max_smem_optin, d->sms, stream);
+    return acc ? launch_gemv_m<false, true>(plan, p, stream)
+               : launch_gemv_m<false, false>(plan, p, stream);
   }
   if (plan.variant == W8A8_VARIANT_GEMM_PAIR) {
     const SplitRegion split = split_region(plan, split_ws, split_ws_bytes);
@@ -891,7 +889,7 @@ int w8a8_linear_fused_ex(const void *x, int64_t M, int64_t K, int64_t ldx, const
     p.ldy = ldy;
     p.q_out = q_out;
     p.s_a_out = s_a_out;
-    return launch_gemv_m<true, false>(plan, p, d->max_smem_optin, d->sms, stream);
+    return launch_gemv_m<true, false>(plan, p, stream);
   }
 
   // workspace layout: [q (M*K) | s_a (M floats) | row-ready counters | K-split region]
