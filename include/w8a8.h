@@ -124,10 +124,11 @@ W8A8_API int w8a8_quantize_weights(const void *W_bf16, int64_t N, int64_t K, int
 
 /*
  * Weight loading from packed int32 storage, run once per layer at load time
- * (the serialized checkpoint form: "Qwen-Image-2.1: TE AutoRound-AWQ on GPU +
- * all-resident single-3090 stack", the quantized-transformer artifact built
- * with pack_to_int32 -- each int8 code stored as an unsigned byte biased by
- * 128, four per int32 word).  packed int32 [N, K/4] dense: word g of row n
+ * (the serialized checkpoint form: "Issue 5 probe: int8 quantized DiT serve
+ * paths on the RTX 3090 (24 GB)", section "Artifact (outside Git, under the
+ * helper state root)": the quantized transformer is packed with
+ * compressed-tensors' pack_to_int32 -- each int8 code stored as an unsigned
+ * byte biased by 128, four per int32 word).  packed int32 [N, K/4] dense: word g of row n
  * holds the codes of columns 4g .. 4g+3, column 4g in the least significant
  * byte -> Wq int8 [N,K] dense, Wq[n,k] = byte - 128.  The per-channel scales
  * s_w are stored beside the packed codes and are used as they are.

@@ -238,9 +238,10 @@ int w8a16_oracle_linear(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
 
 /*
  * The serialized form of an int8 weight: each code stored as an unsigned byte
- * biased by 128, four bytes per int32 word ("Qwen-Image-2.1: TE AutoRound-AWQ
- * on GPU + all-resident single-3090 stack", the artifact description of the
- * quantized transformer built with compressed-tensors' pack_to_int32).  The
+ * biased by 128, four bytes per int32 word ("Issue 5 probe: int8 quantized
+ * DiT serve paths on the RTX 3090 (24 GB)", section "Artifact (outside Git,
+ * under the helper state root)": the quantized transformer is built with
+ * compressed-tensors' pack_to_int32).  The
  * pages fix the bias and the four-per-word ratio; the order inside a word is
  * taken as consecutive codes along K, the first in the least significant
  * byte.  packed is int32 [N][K/4] (K a multiple of 4), Wq int8 [N][K].

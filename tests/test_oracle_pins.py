@@ -388,8 +388,9 @@ def test_planted_wrong_divisor_or_rounding_fails_pin():
 
 # --------------------------------------------------------------------------
 # Packed int32 weight storage: codes biased by 128, four per int32 word
-# ("Qwen-Image-2.1: TE AutoRound-AWQ on GPU + all-resident single-3090 stack",
-# the quantized-transformer artifact built with pack_to_int32).  The order
+# ("Issue 5 probe: int8 quantized DiT serve paths on the RTX 3090 (24 GB)",
+# section "Artifact (outside Git, under the helper state root)": the quantized
+# transformer is built with pack_to_int32).  The order
 # inside a word is a reading: consecutive codes along K, first code in the
 # least significant byte.
 # --------------------------------------------------------------------------
@@ -502,3 +503,187 @@ def test_planted_w8a16_mistakes_fail_pin():
     assert oracle.w8a16_linear(x, wq, np.array([1.0], np.float32))["y32"][0, 0] != 57.0   # scale dropped
     assert oracle.w8a16_linear(x, -wq, np.array([0.5], np.float32))["y32"][0, 0] != 57.0  # sign
     assert oracle.w8a16_linear(x, wq[:, ::-1].copy(), np.array([0.5], np.float32))["y32"][0, 0] != 57.0
+
+
+# --------------------------------------------------------------------------
+# Readings the pages leave open, each fixed by a worked example that a
+# plausible alternative reading gets wrong.  The expected values are derived
+# with exact rational arithmetic and an IEEE round-to-nearest-even written
+# out below (no floating-point arithmetic of numpy, torch or the oracle takes
+# part), and are also stated as literals.
+# --------------------------------------------------------------------------
+
+def rn_binary(v: Fraction, sig_bits: int, emin: int = -126) -> Fraction:
+    """v rounded to the nearest number with `sig_bits` significant bits and
+    minimum normal exponent `emin` (gradual underflow below it), ties to the
+    even significand."""
+    if v == 0:
+        return Fraction(0)
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    quantum = Fraction(2) ** (max(e, emin) - (sig_bits - 1))
+    scaled = a / quantum
+    n = scaled.numerator // scaled.denominator
+    rest = scaled - n
+    if rest > Fraction(1, 2) or (rest == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return sign * n * quantum
+
+
+def rn_f32(v: Fraction) -> Fraction:
+    return rn_binary(v, 24)
+
+
+def rn_bf16(v: Fraction) -> Fraction:
+    return rn_binary(v, 8)
+
+
+def rint_even(v: Fraction) -> int:
+    n = v.numerator // v.denominator
+    rest = v - n
+    if rest > Fraction(1, 2) or (rest == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return n
+
+
+def test_rational_rounding_helper_against_known_values():
+    # the helper itself, on values whose roundings are textbook facts
+    assert rn_f32(Fraction(1, 3)) == Fraction(11184811, 2 ** 25)          # 0x3EAAAAAB
+    assert rn_f32(Fraction(2 ** 24 + 1)) == 2 ** 24                       # tie -> even
+    assert rn_f32(Fraction(2 ** 24 + 3)) == 2 ** 24 + 4                   # tie -> even
+    assert rn_f32(Fraction(1, 2 ** 150)) == 0                             # half the least subnormal: tie -> 0
+    assert rn_f32(Fraction(3, 2 ** 150)) == Fraction(2, 2 ** 149)         # 1.5 subnormal quanta -> 2
+    assert rn_bf16(Fraction(257, 256)) == 1                               # 1 + 2^-8: tie -> 1.0
+    assert rn_bf16(Fraction(259, 256)) == Fraction(260, 256)              # 1 + 3*2^-8: tie -> 1.015625
+    assert rint_even(Fraction(5, 2)) == 2 and rint_even(Fraction(-5, 2)) == -2
+    assert rint_even(Fraction(7, 2)) == 4 and rint_even(Fraction(-1, 2)) == 0
+
+
+# Two rows on which "x divided by the stored fp32 scale" and the reciprocal
+# readings give different codes.  Row A: s = RN(5.59375/127) = 5911657 * 2^-27,
+# 2.796875 / s = 63.49999805... (fp32 quotient 63.499996) -> 63, while
+# x * RN(127/amax), x * RN(1/s) and RN(x*127)/amax all round to 63.5 -> 64.
+# Row B: s = 14861707 * 2^-32; 0.2197265625 / s = 63.50000037... (fp32
+# quotient exactly 63.5) -> 64, while both reciprocal forms give 63.499996 -> 63.
+QUOTIENT_ROWS = [
+    ([5.59375, 2.796875, -2.796875, 1.0], Fraction(5911657, 2 ** 27), [127, 63, -63, 23]),
+    ([0.439453125, 0.2197265625, -0.2197265625, 0.0078125], Fraction(14861707, 2 ** 32),
+     [127, 64, -64, 2]),
+]
+
+
+def _codes(row, quotient):
+    amax = max(abs(Fraction(v)) for v in row)
+    s = rn_f32(amax / 127)
+    return s, [max(-127, min(127, rint_even(quotient(Fraction(v), s, amax)))) for v in row]
+
+
+def _q_divide(x, s, amax):
+    return rn_f32(x / s)
+
+
+def _q_times_127_over_amax(x, s, amax):
+    return rn_f32(x * rn_f32(Fraction(127) / amax))
+
+
+def _q_times_reciprocal_of_s(x, s, amax):
+    return rn_f32(x * rn_f32(1 / s))
+
+
+def _q_scaled_then_divided(x, s, amax):
+    return rn_f32(rn_f32(x * 127) / amax)
+
+
+@pytest.mark.parametrize("row,s_exp,q_exp", QUOTIENT_ROWS)
+def test_quotient_is_ieee_division_by_the_stored_scale(row, s_exp, q_exp):
+    s_def, q_def = _codes(row, _q_divide)
+    assert s_def == s_exp and q_def == q_exp          # the literals follow from the definition
+    q, s = oracle.quant_rows(bits([row]))
+    assert Fraction(float(s[0])) == s_exp
+    assert q[0].tolist() == q_exp
+
+
+@pytest.mark.parametrize("row,s_exp,q_exp", QUOTIENT_ROWS)
+def test_planted_reciprocal_quotients_fail_the_pin(row, s_exp, q_exp):
+    # an oracle that multiplied by a rounded reciprocal would not reproduce q_exp
+    for quotient in (_q_times_127_over_amax, _q_times_reciprocal_of_s):
+        assert _codes(row, quotient)[1] != q_exp, quotient.__name__
+    if row[0] == 5.59375:
+        assert _codes(row, _q_scaled_then_divided)[1] != q_exp
+
+
+# The epilogue is four separately rounded fp32 operations in a fixed order:
+# f = RN((float)acc), p = RN(f * s_a), p = RN(p * s_w), y32 = RN(p + bias),
+# then y = bf16_rne(y32).  Each example lands next to a bf16 tie, so a
+# reordered product, a fused multiply-add or a truncating int -> float
+# conversion changes the bf16 output itself, not only y32.
+#   (acc, s_a bits, s_w bits, bias bf16 bits or None, y32, y)
+EPILOGUE_EXAMPLES = [
+    # f = -54427616 (acc is a tie between -54427620 and -54427616 -> even);
+    # y32 = -67.75 exactly, a bf16 tie -> -68.  Scaling by RN(s_a * s_w), or
+    # by s_w first, gives -67.749992 -> -67.5.
+    (-54427618, 0x3AF2C7C0, 0x3A30294F, 0xBB21, Fraction(-271, 4), Fraction(-68)),
+    # y32 = 425.0, a bf16 tie -> 424.  A fused multiply-add of the bias gives
+    # 425.00003 -> 426.
+    (60900663, 0x3C2FD9E8, 0x3A2A71C1, 0xBA96, Fraction(425), Fraction(424)),
+    # f = 39177160 (nearest); y32 = 1620.0001220703125 -> 1624.  Converting
+    # acc by truncation (39177156) gives 1619.99988 -> 1616.
+    (39177159, 0x3CFA7FFC, 0x3AB13EC2, None, Fraction(1620) + Fraction(1, 8192), Fraction(1624)),
+]
+
+
+def _u32_to_fraction(u):
+    return Fraction(float(np.array([u], np.uint32).view(np.float32)[0]))
+
+
+def _bf16_bits_to_fraction(b):
+    return Fraction(float(f64(np.array([b], np.uint16))[0]))
+
+
+def _epilogue_def(acc, sa, sw, b, order="definition"):
+    f = rn_f32(Fraction(acc))
+    if order == "truncating_conversion":
+        q = Fraction(2) ** (abs(acc).bit_length() - 24)
+        f = Fraction(int(Fraction(acc) / q) * q) if abs(acc) >= 2 ** 24 else Fraction(acc)
+    if order == "prescaled":
+        p = rn_f32(f * rn_f32(sa * sw))
+    elif order == "swapped":
+        p = rn_f32(rn_f32(f * sw) * sa)
+    else:
+        p = rn_f32(rn_f32(f * sa) * sw)
+    if b is None:
+        return p
+    if order == "fma":
+        return rn_f32(rn_f32(f * sa) * sw + b)
+    return rn_f32(p + b)
+
+
+@pytest.mark.parametrize("acc,sa_u,sw_u,b_u,y32_exp,y_exp", EPILOGUE_EXAMPLES)
+def test_epilogue_order_worked_examples(acc, sa_u, sw_u, b_u, y32_exp, y_exp):
+    sa, sw = _u32_to_fraction(sa_u), _u32_to_fraction(sw_u)
+    b = None if b_u is None else _bf16_bits_to_fraction(b_u)
+    y32_def = _epilogue_def(acc, sa, sw, b)
+    assert y32_def == y32_exp and rn_bf16(y32_def) == y_exp
+    s_a = np.array([sa_u], np.uint32).view(np.float32)
+    s_w = np.array([sw_u], np.uint32).view(np.float32)
+    bias = None if b_u is None else np.array([b_u], np.uint16)
+    y32, y = oracle.epilogue(np.array([[acc]], np.int32), s_a, s_w, bias)
+    assert Fraction(float(y32[0, 0])) == y32_exp
+    assert _bf16_bits_to_fraction(int(y[0, 0])) == y_exp
+
+
+def test_planted_epilogue_orders_fail_the_pin():
+    # every alternative order changes the bf16 output of at least one example
+    for order in ("prescaled", "swapped", "fma", "truncating_conversion"):
+        changed = False
+        for acc, sa_u, sw_u, b_u, _, y_exp in EPILOGUE_EXAMPLES:
+            sa, sw = _u32_to_fraction(sa_u), _u32_to_fraction(sw_u)
+            b = None if b_u is None else _bf16_bits_to_fraction(b_u)
+            if rn_bf16(_epilogue_def(acc, sa, sw, b, order)) != y_exp:
+                changed = True
+        assert changed, order

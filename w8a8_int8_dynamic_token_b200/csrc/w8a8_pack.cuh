@@ -1,9 +1,10 @@
 // w8a8_pack.cuh -- loading int8 weights from their packed int32 storage.
 //
 // A serialized W8A8 checkpoint stores each int8 weight code as an unsigned
-// byte biased by 128, four per int32 word ("Qwen-Image-2.1: TE AutoRound-AWQ
-// on GPU + all-resident single-3090 stack", the quantized-transformer
-// artifact built with compressed-tensors' pack_to_int32).  Codes run along K,
+// byte biased by 128, four per int32 word ("Issue 5 probe: int8 quantized DiT
+// serve paths on the RTX 3090 (24 GB)", section "Artifact (outside Git, under
+// the helper state root)": the quantized transformer is built with
+// compressed-tensors' pack_to_int32).  Codes run along K,
 // the first of each group of four in the least significant byte, so on a
 // little-endian device the packed array's bytes, in memory order, are
 // (code + 128) mod 256 = code XOR 0x80: unpacking is a byte-wise XOR that
