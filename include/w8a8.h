@@ -152,9 +152,11 @@ W8A8_API int w8a8_quant_act(const void *x_bf16, int64_t M, int64_t K, int64_t ld
  * activations and their scales, one 64-bit counter per 128 rows (used by
  * the one-launch option of w8a8_linear_fused_ex), plus, when the plan shares
  * its last tiles out along K (w8a8_plan.split_tiles > 0), the int32 partial
- * sums and arrival counters of that region.  Nothing in it needs
- * initializing.  A workspace holding only q and s_a still works: the layer
- * then runs without the K split.
+ * sums and arrival counters of that region.  The caller need not initialize
+ * it: a call that uses counters clears them on its stream first (an
+ * asynchronous memset of a few KB; nothing is allocated).  A workspace
+ * holding only q and s_a still works: the layer then runs without the K
+ * split.
  */
 W8A8_API int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes);
 
@@ -166,9 +168,11 @@ W8A8_API int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes)
  * accumulators are written there INSTEAD of y (y may then be NULL).
  * workspace / ws_bytes: optional (NULL / 0 allowed).  With at least
  * w8a8_workspace_size(M,N,K) bytes (16-byte aligned) the pair kernel's K-split
- * tail is used.  Its contents need no initialization (arrival counters carry
- * a per-launch tag and are reset by the kernel); the workspace must not be in
- * use by other work while the call runs.  After a launch that reported
+ * tail is used.  Its contents need no initialization: the call clears the
+ * region's arrival counters on `stream` before the launch, and the counters
+ * also carry a per-launch tag drawn from a random per-process start, so
+ * words another launch left behind count as zero.  The workspace must not
+ * be in use by other work while the call runs.  After a launch that reported
  * W8A8_ERR_DEVICE_TIMEOUT, replaying a captured graph of it on the same
  * workspace is outside the contract.
  */
@@ -318,6 +322,15 @@ W8A8_API int w8a8_linear_fused_noalloc(const void *x_bf16, int64_t M, int64_t K,
  * on the order of a second.
  */
 W8A8_API int w8a8_selftest_quant_exhaustive(unsigned long long *counts_dev, w8a8_stream_t stream);
+
+/*
+ * Test support: the launch tag that the next call using arrival counters
+ * (a K-split tail, or the one-launch option of w8a8_linear_fused_ex) will
+ * draw, in its low 56 bits (the one-launch option uses the low 48).  A test
+ * can plant a counter word carrying this tag in a workspace and check that
+ * the call still computes the right result.  Host-only; needs no GPU.
+ */
+W8A8_API int w8a8_debug_peek_tag(uint64_t *tag);
 
 /* Library version string, e.g. "w8a8 1.0 sm_100a". */
 W8A8_API const char *w8a8_version(void);

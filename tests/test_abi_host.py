@@ -305,3 +305,48 @@ def test_selector_plans_are_valid_for_random_shapes(M, n8, k16):
         assert (tiles - st) % pairs == 0
     if p["quant_in_gemm_launch"]:
         assert K <= 3072 and _cdiv(M, p["grid"] * 8) <= 4
+
+
+# --------------------------------------------------------------------------
+# The torch binding checks shapes before anything reaches the library: a
+# short bias or output would otherwise let a kernel read or write past the
+# end of a buffer.
+# --------------------------------------------------------------------------
+
+def _cpu_layer(M=8, N=16, K=32):
+    import torch
+    return (torch.zeros((M, K), dtype=torch.bfloat16), torch.zeros((N, K), dtype=torch.int8),
+            torch.ones(N, dtype=torch.float32))
+
+
+@pytest.mark.parametrize("fn", ["linear_fused", "w8a16_linear"])
+def test_binding_rejects_short_bias_and_output(fn):
+    import torch
+    x, Wq, s_w = _cpu_layer()
+    call = getattr(w8a8, fn)
+    with pytest.raises(ValueError, match="bias must have shape"):
+        call(x, Wq, s_w, torch.zeros(15, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="out must have shape"):
+        call(x, Wq, s_w, None, out=torch.zeros((7, 16), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="out must have shape"):
+        # fewer rows than M, however wide its row stride
+        call(x, Wq, s_w, None, out=torch.zeros((7, 64), dtype=torch.bfloat16)[:, :16])
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        call(x, Wq, s_w, torch.zeros(16, dtype=torch.bfloat16))   # shapes fine: device next
+
+
+def test_binding_linear_rejects_short_bias_and_output():
+    import torch
+    q = torch.zeros((8, 32), dtype=torch.int8)
+    s_a = torch.ones(8, dtype=torch.float32)
+    _, Wq, s_w = _cpu_layer()
+    with pytest.raises(ValueError, match="bias must have shape"):
+        w8a8.linear(q, s_a, Wq, s_w, torch.zeros(8, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="out must have shape"):
+        w8a8.linear(q, s_a, Wq, s_w, out=torch.zeros((8, 8), dtype=torch.bfloat16))
+
+
+def test_debug_peek_tag_is_stable_without_launches():
+    a = B.debug_peek_tag()
+    b = B.debug_peek_tag()
+    assert a == b and 0 < a < 2 ** 56

@@ -305,7 +305,7 @@ def test_ffn_pair_back_to_back():
         assert check_y(bits_of(y)[rows], y_ref, y32, "ffn pair") == 0
 
 
-SWEEP = [c for c in synth.sweep_cases() if c.seed == 0 or c.M <= 4352]
+SWEEP = synth.sweep_cases()
 
 
 @pytest.mark.parametrize("case", SWEEP, ids=lambda c: c.name)
@@ -471,6 +471,33 @@ def test_pair_k_split_repeated_calls_on_one_workspace():
     for i, (q, acc) in enumerate(zip(qs, accs)):
         rows = sample_rows(M, seed=i, n_random=16, tile=256)
         assert np.array_equal(acc.cpu().numpy()[rows], oracle.gemm_i32(q[rows], wq)), i
+
+
+def test_pair_k_split_ignores_counter_words_planted_with_the_live_tag():
+    """A workspace whose every 64-bit word reads as a counter of the very
+    launch about to run, with all but one contribution already arrived
+    ((tag << 8) | 3 for tiles shared by four pairs): without the clearing
+    before the launch, the first contribution to arrive would finish its tile
+    from partial sums nobody wrote.  The result must still equal the unsplit
+    kernel and the oracle."""
+    M, N, K = 512, 1024, 12288
+    assert w8a8.select(M, N, K, variant=B.VARIANT_GEMM_PAIR)["split_tiles"] > 0
+    rng = np.random.default_rng(123)
+    q = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
+    wq = rng.integers(-127, 128, size=(N, K), dtype=np.int8)
+    args = (torch.from_numpy(q).cuda(), torch.ones(M, device="cuda"), torch.from_numpy(wq).cuda(),
+            torch.ones(N, device="cuda"))
+    ref_plain = w8a8.linear(*args, acc_debug=True, variant=B.VARIANT_GEMM_PAIR, split=False)
+    ws = torch.empty((w8a8.workspace_size(M, N, K),), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        torch.cuda.synchronize()
+        word = np.array([(B.debug_peek_tag() << 8) | 3], dtype=np.uint64).view(np.int64)[0]
+        ws.view(torch.int64).fill_(int(word))
+        acc = w8a8.linear(*args, acc_debug=True, variant=B.VARIANT_GEMM_PAIR, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(acc, ref_plain)
+    rows = sample_rows(M, seed=5, n_random=16, tile=256)
+    assert np.array_equal(acc.cpu().numpy()[rows], oracle.gemm_i32(q[rows], wq))
 
 
 # ----------------------------------------------------------------- packed weights

@@ -70,7 +70,7 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls(M, N, K):
         rows = sample_rows(M, seed=call, n_random=32)
         q_ref, s_ref = oracle.quant_rows(x_bits[rows])
         y32, y_ref = oracle.epilogue(oracle.gemm_i32(q_ref, wq_ref), s_ref, sw_ref, b_bits)
-        check_y(bits_of(y_static)[rows], y_ref, y32, f"noalloc call {call}")
+        assert check_y(bits_of(y_static)[rows], y_ref, y32, f"noalloc call {call}") == 0
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():

@@ -12,6 +12,7 @@ or PyTorch fallback: if libw8a8.so is missing this module raises on first use.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import functools
 import os
@@ -87,6 +88,7 @@ _SIGNATURES = {
     "w8a8_last_device_error": ([_vp], _int),
     "w8a8_selftest_bounded_wait": ([_i64, _vp], _int),
     "w8a8_selftest_quant_exhaustive": ([_vp, _vp], _int),
+    "w8a8_debug_peek_tag": ([ctypes.POINTER(ctypes.c_uint64)], _int),
 }
 
 
@@ -213,19 +215,55 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _need(t, name, dtype, ndim, device=None):
+def _need(t, name, dtype, ndim):
+    """dtype, rank and unit inner stride (checked before the device, so shape
+    errors surface the same way on any device)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if t.dim() != ndim:
         raise ValueError(f"{name} must be {ndim}-D")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
-    if device is not None and t.device != device:
-        raise ValueError(f"{name} is on {t.device}, expected {device}")
-    if t.stride(-1) != 1:
+    if t.numel() > 0 and t.stride(-1) != 1:
         raise ValueError(f"{name} must have unit stride in its last dimension")
+
+
+def _shape(t, name, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _on_one_device(**tensors):
+    """The CUDA device every given tensor lives on (all must share it)."""
+    dev = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    return dev
+
+
+@contextlib.contextmanager
+def _launching(dev, stream=None):
+    """Run a call on the tensors' device: the library reads the current device
+    (its properties, and the allocation-free scratch), so that device is made
+    current.  The call is enqueued on `stream`, or on that device's current
+    stream; tensors allocated inside belong to that stream, so the caching
+    allocator never hands their memory to other work while the call may still
+    use it."""
+    with torch.cuda.device(dev):
+        if stream is None:
+            yield torch.cuda.current_stream()
+        else:
+            if stream.device != dev:
+                raise ValueError(f"stream is on {stream.device}, the tensors on {dev}")
+            with torch.cuda.stream(stream):
+                yield stream
 
 
 @functools.lru_cache(maxsize=1024)
@@ -246,11 +284,13 @@ def select(M: int, N: int, K: int, num_sms: int = 148, variant: int = VARIANT_AU
 def quantize_weights(W: torch.Tensor, stream=None):
     """bf16 W [N, K] -> (Wq int8 [N, K], s_w fp32 [N]) on W's device."""
     _need(W, "W", torch.bfloat16, 2)
+    dev = _on_one_device(W=W)
     N, K = W.shape
-    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
-    s_w = torch.empty((N,), dtype=torch.float32, device=W.device)
-    _check(w8a8_quantize_weights(_ptr(W), N, K, W.stride(0), _ptr(Wq), _ptr(s_w),
-                                 _stream(stream)), "w8a8_quantize_weights")
+    with _launching(dev, stream) as s:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        s_w = torch.empty((N,), dtype=torch.float32, device=dev)
+        _check(w8a8_quantize_weights(_ptr(W), N, K, W.stride(0), _ptr(Wq), _ptr(s_w), _stream(s)),
+               "w8a8_quantize_weights")
     return Wq, s_w
 
 
@@ -260,30 +300,35 @@ def unpack_int32_weights(packed: torch.Tensor, stream=None) -> torch.Tensor:
     _need(packed, "packed", torch.int32, 2)
     if not packed.is_contiguous():
         raise ValueError("packed must be dense row-major")
+    dev = _on_one_device(packed=packed)
     N, K = packed.shape[0], packed.shape[1] * 4
-    Wq = torch.empty((N, K), dtype=torch.int8, device=packed.device)
-    _check(w8a8_unpack_int32_weights(_ptr(packed), N, K, _ptr(Wq), _stream(stream)),
-           "w8a8_unpack_int32_weights")
+    with _launching(dev, stream) as s:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        _check(w8a8_unpack_int32_weights(_ptr(packed), N, K, _ptr(Wq), _stream(s)),
+               "w8a8_unpack_int32_weights")
     return Wq
 
 
 def quant_act(x: torch.Tensor, stream=None):
     """bf16 x [M, K] -> (q int8 [M, K], s_a fp32 [M])."""
     _need(x, "x", torch.bfloat16, 2)
+    dev = _on_one_device(x=x)
     M, K = x.shape
-    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
-    s_a = torch.empty((M,), dtype=torch.float32, device=x.device)
-    _check(w8a8_quant_act(_ptr(x), M, K, x.stride(0), _ptr(q), _ptr(s_a), _stream(stream)),
-           "w8a8_quant_act")
+    with _launching(dev, stream) as s:
+        q = torch.empty((M, K), dtype=torch.int8, device=dev)
+        s_a = torch.empty((M,), dtype=torch.float32, device=dev)
+        _check(w8a8_quant_act(_ptr(x), M, K, x.stride(0), _ptr(q), _ptr(s_a), _stream(s)),
+               "w8a8_quant_act")
     return q, s_a
 
 
 def _workspace_for(M, N, K, workspace, dev):
     """(tensor, pointer, bytes): the caller's workspace, or a fresh one of
-    workspace_size(M, N, K) bytes when `workspace` is None.  The caller keeps
-    the returned tensor alive until the launch has been enqueued: the device
-    memory must not return to the allocator before then, or an output
-    allocated afterwards could share it."""
+    workspace_size(M, N, K) bytes when `workspace` is None (allocated on the
+    launching stream, inside _launching).  The caller keeps the returned
+    tensor alive until the launch has been enqueued: the device memory must
+    not return to the allocator before then, or an output allocated
+    afterwards could share it."""
     need = workspace_size(M, N, K)
     if workspace is None:
         if need == 0:
@@ -292,41 +337,48 @@ def _workspace_for(M, N, K, workspace, dev):
     return workspace, _ptr(workspace), workspace.numel() * workspace.element_size()
 
 
+def _check_layer_args(M, N, K, bias, out):
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+        _shape(bias, "bias", (N,))
+    if out is not None:
+        _need(out, "out", torch.bfloat16, 2)
+        _shape(out, "out", (M, N))
+
+
 def linear(q, s_a, Wq, s_w, bias=None, out=None, acc_debug=False, variant=VARIANT_AUTO,
            workspace=None, split=True, stream=None):
     """y = bf16(((float)(q @ Wq^T) * s_a) * s_w + bias); with acc_debug=True the raw
     int32 accumulators [M, N] are returned instead.  split=False runs the pair
     kernel without its K-split tail (no workspace is passed)."""
     _need(q, "q", torch.int8, 2)
-    dev = q.device
-    _need(s_a, "s_a", torch.float32, 1, dev)
-    _need(Wq, "Wq", torch.int8, 2, dev)
-    _need(s_w, "s_w", torch.float32, 1, dev)
+    _need(s_a, "s_a", torch.float32, 1)
+    _need(Wq, "Wq", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
     M, K = q.shape
     N = Wq.shape[0]
     if Wq.shape[1] != K or s_a.shape[0] != M or s_w.shape[0] != N:
         raise ValueError("shape mismatch between q, s_a, Wq, s_w")
     if not (q.is_contiguous() and Wq.is_contiguous()):
         raise ValueError("q and Wq must be dense row-major")
-    if bias is not None:
-        _need(bias, "bias", torch.bfloat16, 1, dev)
-        if bias.shape[0] != N:
-            raise ValueError("bias must have N elements")
-    ws, ws_ptr, ws_bytes = (_workspace_for(M, N, K, workspace, dev) if split
-                            else (None, None, 0))
-    if acc_debug:
-        acc = torch.empty((M, N), dtype=torch.int32, device=dev)
+    _check_layer_args(M, N, K, bias, None if acc_debug else out)
+    dev = _on_one_device(q=q, s_a=s_a, Wq=Wq, s_w=s_w, bias=bias,
+                         out=None if acc_debug else out, workspace=workspace)
+    with _launching(dev, stream) as s:
+        ws, ws_ptr, ws_bytes = (_workspace_for(M, N, K, workspace, dev) if split
+                                else (None, None, 0))
+        if acc_debug:
+            acc = torch.empty((M, N), dtype=torch.int32, device=dev)
+            _check(w8a8_linear_ex(_ptr(q), _ptr(s_a), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
+                                  None, N, _ptr(acc), variant, ws_ptr, ws_bytes, _stream(s)),
+                   "w8a8_linear_ex")
+            del ws  # enqueued on s: later allocations on s are ordered after the launch
+            return acc
+        y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         _check(w8a8_linear_ex(_ptr(q), _ptr(s_a), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
-                              None, N, _ptr(acc), variant, ws_ptr, ws_bytes, _stream(stream)),
+                              _ptr(y), y.stride(0), None, variant, ws_ptr, ws_bytes, _stream(s)),
                "w8a8_linear_ex")
-        del ws  # enqueued: later allocations on this stream are ordered after the launch
-        return acc
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    _need(y, "out", torch.bfloat16, 2, dev)
-    _check(w8a8_linear_ex(_ptr(q), _ptr(s_a), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
-                          _ptr(y), y.stride(0), None, variant, ws_ptr, ws_bytes,
-                          _stream(stream)), "w8a8_linear_ex")
-    del ws
+        del ws
     return y
 
 
@@ -335,25 +387,25 @@ def linear_fused(x, Wq, s_w, bias=None, out=None, workspace=None, return_interme
     """Whole layer from bf16 x [M, K]: per-token quantization, int8 GEMM, fused
     epilogue.  Returns y [M, N] (and (q, s_a) with return_intermediates=True)."""
     _need(x, "x", torch.bfloat16, 2)
-    dev = x.device
-    _need(Wq, "Wq", torch.int8, 2, dev)
-    _need(s_w, "s_w", torch.float32, 1, dev)
+    _need(Wq, "Wq", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
     M, K = x.shape
     N = Wq.shape[0]
     if Wq.shape[1] != K or s_w.shape[0] != N or not Wq.is_contiguous():
         raise ValueError("shape mismatch between x, Wq, s_w")
-    if bias is not None:
-        _need(bias, "bias", torch.bfloat16, 1, dev)
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    _need(y, "out", torch.bfloat16, 2, dev)
-    q = s_a = None
-    if return_intermediates:
-        q = torch.empty((M, K), dtype=torch.int8, device=dev)
-        s_a = torch.empty((M,), dtype=torch.float32, device=dev)
-    ws, ws_ptr, ws_bytes = _workspace_for(M, N, K, workspace, dev)
-    _check(w8a8_linear_fused(_ptr(x), M, K, x.stride(0), _ptr(Wq), _ptr(s_w), _ptr(bias), N,
-                             _ptr(y), y.stride(0), _ptr(q), _ptr(s_a), ws_ptr, ws_bytes,
-                             _stream(stream)), "w8a8_linear_fused")
+    _check_layer_args(M, N, K, bias, out)
+    dev = _on_one_device(x=x, Wq=Wq, s_w=s_w, bias=bias, out=out, workspace=workspace)
+    with _launching(dev, stream) as s:
+        y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        q = s_a = None
+        if return_intermediates:
+            q = torch.empty((M, K), dtype=torch.int8, device=dev)
+            s_a = torch.empty((M,), dtype=torch.float32, device=dev)
+        ws, ws_ptr, ws_bytes = _workspace_for(M, N, K, workspace, dev)
+        _check(w8a8_linear_fused(_ptr(x), M, K, x.stride(0), _ptr(Wq), _ptr(s_w), _ptr(bias), N,
+                                 _ptr(y), y.stride(0), _ptr(q), _ptr(s_a), ws_ptr, ws_bytes,
+                                 _stream(s)), "w8a8_linear_fused")
+        del ws
     if return_intermediates:
         return y, q, s_a
     return y
@@ -363,19 +415,18 @@ def w8a16_linear(x, Wq, s_w, bias=None, out=None, stream=None):
     """Weight-only int8 layer on bf16 x [M, K]: y = bf16((x @ Wq^T) * s_w + bias),
     fp32 accumulation on the tensor cores."""
     _need(x, "x", torch.bfloat16, 2)
-    dev = x.device
-    _need(Wq, "Wq", torch.int8, 2, dev)
-    _need(s_w, "s_w", torch.float32, 1, dev)
+    _need(Wq, "Wq", torch.int8, 2)
+    _need(s_w, "s_w", torch.float32, 1)
     M, K = x.shape
     N = Wq.shape[0]
     if Wq.shape[1] != K or s_w.shape[0] != N or not Wq.is_contiguous():
         raise ValueError("shape mismatch between x, Wq, s_w")
-    if bias is not None:
-        _need(bias, "bias", torch.bfloat16, 1, dev)
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    _need(y, "out", torch.bfloat16, 2, dev)
-    _check(w8a16_linear_raw(_ptr(x), M, K, x.stride(0), _ptr(Wq), _ptr(s_w), _ptr(bias), N,
-                            _ptr(y), y.stride(0), _stream(stream)), "w8a16_linear")
+    _check_layer_args(M, N, K, bias, out)
+    dev = _on_one_device(x=x, Wq=Wq, s_w=s_w, bias=bias, out=out)
+    with _launching(dev, stream) as s:
+        y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        _check(w8a16_linear_raw(_ptr(x), M, K, x.stride(0), _ptr(Wq), _ptr(s_w), _ptr(bias), N,
+                                _ptr(y), y.stride(0), _stream(s)), "w8a16_linear")
     return y
 
 
@@ -384,10 +435,14 @@ def linear_fused_host(x_host, Wq, s_w, bias, y_host, x_dev, y_dev, workspace, st
     (all enqueued on the stream; synchronize before reading y_host)."""
     M, K = x_host.shape
     N = Wq.shape[0]
+    if tuple(y_host.shape) != (M, N) or tuple(x_dev.shape) != (M, K) or tuple(y_dev.shape) != (M, N):
+        raise ValueError("x_host / x_dev must be [M, K] and y_host / y_dev [M, N]")
+    dev = _on_one_device(Wq=Wq, s_w=s_w, bias=bias, x_dev=x_dev, y_dev=y_dev, workspace=workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(w8a8_linear_fused_host(_ptr(x_host), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
-                                  _ptr(y_host), _ptr(x_dev), _ptr(y_dev), _ptr(workspace),
-                                  ws_bytes, _stream(stream)), "w8a8_linear_fused_host")
+    with _launching(dev, stream) as s:
+        _check(w8a8_linear_fused_host(_ptr(x_host), M, K, _ptr(Wq), _ptr(s_w), _ptr(bias), N,
+                                      _ptr(y_host), _ptr(x_dev), _ptr(y_dev), _ptr(workspace),
+                                      ws_bytes, _stream(s)), "w8a8_linear_fused_host")
     return y_host
 
 
@@ -411,3 +466,10 @@ def selftest_quant_exhaustive(stream=None) -> tuple[int, int]:
     torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
     c = counts.cpu().tolist()
     return int(c[0]), int(c[1])
+
+
+def debug_peek_tag() -> int:
+    """The launch tag the next call using arrival counters will draw."""
+    out = ctypes.c_uint64(0)
+    _check(lib().w8a8_debug_peek_tag(ctypes.byref(out)), "w8a8_debug_peek_tag")
+    return int(out.value)

@@ -7,9 +7,11 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <chrono>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <random>
 
 #include "../../include/w8a8.h"
 #include "w8a8_gemm.cuh"
@@ -240,7 +242,8 @@ size_t fused_workspace_bytes(int64_t M, int64_t K) {
 
 // The pair kernel's K-split region: arrival counters (16 per shared-out
 // tile, 64-bit), then the partial-sum slots (split_tiles + pairs - 1 of them,
-// 16 slices of 32 x 128 int32 each).  Nothing in it needs initializing.
+// 16 slices of 32 x 128 int32 each).  The counters are cleared on the stream
+// before each launch that uses them; the partial sums need no initializing.
 size_t split_counter_bytes(const w8a8_plan &plan) {
   return align256(static_cast<size_t>(plan.split_tiles) * kSlicesPerTile *
                   sizeof(unsigned long long));
@@ -258,10 +261,42 @@ struct SplitRegion {
   int32_t *partials = nullptr;
 };
 
-// Launch tags of the K-split arrival counters: distinct for every launch of
-// the process (a captured graph replays its tag; the counters it leaves are
-// reset to 0, which no tag equals).
-std::atomic<unsigned long long> g_split_epoch{1};
+// Launch tags of the arrival counters (K-split tail, fused quantization).
+// The host clears a launch's counter region (cudaMemsetAsync, which
+// allocates nothing) before the launch, and every counter also carries the
+// launch's tag, so a word that some other launch left counts as zero.  Tags
+// count up from a random start drawn once per process: memory written by
+// other code (another layer's activations, another process's counters) is
+// not mistaken for a live counter except by a 2^-48 chance.
+unsigned long long initial_tag() {
+  unsigned long long t = 0;
+  try {
+    std::random_device rd;
+    t = (static_cast<unsigned long long>(rd()) << 32) ^ rd();
+  } catch (...) {
+    t = static_cast<unsigned long long>(
+        std::chrono::high_resolution_clock::now().time_since_epoch().count());
+  }
+  return t;
+}
+std::atomic<unsigned long long> g_tag{initial_tag()};
+
+// The next launch tag, `bits` wide and never 0.
+unsigned long long next_tag(int bits) {
+  const unsigned long long mask = (1ull << bits) - 1;
+  const unsigned long long t = g_tag.fetch_add(1, std::memory_order_relaxed) & mask;
+  return t != 0 ? t : 1;
+}
+
+// Clears `bytes` of counters on `stream` before the launch that uses them.
+int clear_counters(void *p, size_t bytes, cudaStream_t stream) {
+  if (p == nullptr || bytes == 0) return W8A8_OK;
+  if (cudaMemsetAsync(p, 0, bytes, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  return W8A8_OK;
+}
 
 SplitRegion split_region(const w8a8_plan &plan, void *base, size_t bytes) {
   SplitRegion r;
@@ -552,8 +587,7 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
     p.sk_units = plan.split_tiles * p.k_blocks;
     p.split_partials = split.partials;
     p.split_counters = split.counters;
-    p.split_epoch = g_split_epoch.fetch_add(1, std::memory_order_relaxed) & kSplitEpochMask;
-    if (p.split_epoch == 0) p.split_epoch = 1;
+    p.split_epoch = next_tag(56);
   } else if (plan.split_tiles > 0 && plan.num_tiles < plan.grid / 2) {
     grid = 2 * plan.num_tiles;  // unsplit and under one wave: one pair per tile
   }
@@ -569,8 +603,7 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
     p.q_w = const_cast<int8_t *>(q);
     p.s_a_w = const_cast<float *>(s_a);
     p.row_ready = fuse->row_ready;
-    p.fuse_tag = g_split_epoch.fetch_add(1, std::memory_order_relaxed) & ((1ull << 48) - 1);
-    if (p.fuse_tag == 0) p.fuse_tag = 1;
+    p.fuse_tag = next_tag(48);
   }
   constexpr auto kernel = gemm_i8_tcgen05_pair_kernel<kGemmStagesPair, RAW, FUSE>;
   st = ensure_smem_limit<kernel>(L::kSmemBytes);
@@ -631,11 +664,13 @@ __global__ void __launch_bounds__(256) quant_exhaustive_kernel(unsigned long lon
 }
 
 // split_ws / split_ws_bytes: room for the pair kernel's K-split region, or
-// nullptr / 0 (the pair kernel then runs unsplit).
+// nullptr / 0 (the pair kernel then runs unsplit).  counters_cleared: the
+// caller has already cleared the region's counters on `stream` (before an
+// earlier launch of the same call), so none is issued here.
 int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
                 const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
                 int32_t *acc, int variant, void *split_ws, size_t split_ws_bytes,
-                cudaStream_t stream) {
+                bool counters_cleared, cudaStream_t stream) {
   if (!q || !s_a || !Wq || !s_w || (!y && !acc)) return W8A8_ERR_INVALID_ARG;
   int st = check_mk(M, K, K);
   if (st != W8A8_OK) return st;
@@ -669,6 +704,10 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
   }
   if (plan.variant == W8A8_VARIANT_GEMM_PAIR) {
     const SplitRegion split = split_region(plan, split_ws, split_ws_bytes);
+    if (!counters_cleared) {
+      st = clear_counters(split.counters, split.counters ? split_counter_bytes(plan) : 0, stream);
+      if (st != W8A8_OK) return st;
+    }
     return acc ? launch_gemm_pair<true, false>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc,
                                                split, nullptr, stream)
                : launch_gemm_pair<false, false>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc,
@@ -756,7 +795,14 @@ const char *w8a8_status_string(int status) {
   }
 }
 
-const char *w8a8_version(void) { return "w8a8 1.0 sm_100a"; }
+const char *w8a8_version(void) { return "w8a8 1.1 sm_100a"; }
+
+int w8a8_debug_peek_tag(uint64_t *tag) {
+  if (!tag) return W8A8_ERR_INVALID_ARG;
+  const unsigned long long t = g_tag.load(std::memory_order_relaxed) & ((1ull << 56) - 1);
+  *tag = t != 0 ? t : 1;
+  return W8A8_OK;
+}
 
 int w8a8_quantize_weights(const void *W, int64_t N, int64_t K, int64_t ldw, int8_t *Wq,
                           float *s_w, w8a8_stream_t stream) {
@@ -832,7 +878,7 @@ int w8a8_linear(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
                 const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
                 int32_t *acc_debug, void *workspace, size_t ws_bytes, w8a8_stream_t stream) {
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, W8A8_VARIANT_AUTO,
-                     workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+                     workspace, ws_bytes, false, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K, const int8_t *Wq,
@@ -842,7 +888,7 @@ int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K, cons
   if (variant < W8A8_VARIANT_AUTO || variant > W8A8_VARIANT_GEMM_BN64)
     return W8A8_ERR_INVALID_ARG;
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant, workspace,
-                     ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+                     ws_bytes, false, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_linear_fused(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t *Wq,
@@ -910,11 +956,11 @@ int w8a8_linear_fused_ex(const void *x, int64_t M, int64_t K, int64_t ldx, const
     split_ws = static_cast<uint8_t *>(workspace) + head;
     split_bytes = ws_bytes - head;
   }
-  // One launch only on request: measured slower than the two launches (the
-  // epilogue warps alone quantize with too little memory parallelism; see the
-  // design notes).  Its counters carry a tag drawn here, on the host: a
-  // captured graph would replay one tag, so under stream capture the two
-  // launches are used instead.
+  // One launch only on request: it measured 6-17% slower than the two
+  // launches, because the 8 epilogue warps of a CTA, quantizing before the
+  // first tiles, keep too few loads in flight to stream x at HBM speed.  Its
+  // counters carry a tag drawn here, on the host: a captured graph would
+  // replay one tag, so under stream capture the two launches are used instead.
   cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
   if ((options & W8A8_FUSED_ONE_LAUNCH) && cudaStreamIsCapturing(stream, &capture) != cudaSuccess) {
     cudaGetLastError();
@@ -930,13 +976,24 @@ int w8a8_linear_fused_ex(const void *x, int64_t M, int64_t K, int64_t ldx, const
     f.row_ready = reinterpret_cast<unsigned long long *>(static_cast<uint8_t *>(workspace) +
                                                          qs_bytes);
     const SplitRegion split = split_region(plan, split_ws, split_bytes);
+    st = clear_counters(f.row_ready, ready_counter_bytes(M), stream);
+    if (st != W8A8_OK) return st;
+    st = clear_counters(split.counters, split.counters ? split_counter_bytes(plan) : 0, stream);
+    if (st != W8A8_OK) return st;
     return launch_gemm_pair<false, true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, nullptr,
                                          split, &f, stream);
+  }
+  // the K-split counters are cleared before the quantization kernel, so
+  // that the GEMM stays its programmatic dependent
+  if (plan.variant == W8A8_VARIANT_GEMM_PAIR) {
+    const SplitRegion split = split_region(plan, split_ws, split_bytes);
+    st = clear_counters(split.counters, split.counters ? split_counter_bytes(plan) : 0, stream);
+    if (st != W8A8_OK) return st;
   }
   st = launch_quant(x, M, K, ldx, q, s_a, stream);
   if (st != W8A8_OK) return st;
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, nullptr, plan.variant, split_ws,
-                     split_bytes, stream);
+                     split_bytes, true, stream);
 }
 
 int w8a8_linear_fused_noalloc(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t *Wq,

@@ -91,9 +91,10 @@ struct GemmParams {
   int32_t sk_per;          // K split: units per pair, 0 = no K split
   int32_t sk_units;        // (num_tiles - dp_tiles) * k_blocks
   int32_t *split_partials; // (num_tiles - dp_tiles + pairs - 1) slots of 16 slices
-  // (num_tiles - dp_tiles) x 16 counters, each (tag << 8) | arrivals.  A
-  // counter whose tag is not this launch's split_epoch counts as 0, so the
-  // memory needs no clearing; the electing contribution resets it to 0.
+  // (num_tiles - dp_tiles) x 16 counters, each (tag << 8) | arrivals,
+  // cleared by the host before the launch.  A counter whose tag is not this
+  // launch's split_epoch counts as 0 as well; the electing contribution
+  // resets it to 0.
   unsigned long long *split_counters;
   unsigned long long split_epoch;  // 1 .. 2^56 - 1
   // CTA-pair kernel with the per-token quantization fused in (K <= 3072: a
@@ -102,9 +103,10 @@ struct GemmParams {
   // the buffers the GEMM then reads through tmap_a and s_a.  In pass j, CTA c
   // takes rows 8 c .. 8 c + 7 + j * 8 * gridDim.x (one per epilogue warp), so
   // the 128-row blocks complete in order; after each pass one thread of the
-  // CTA adds its rows to the block's counter, (fuse_tag << 16) | rows (a
-  // counter holding another launch's tag counts as 0: nothing needs
-  // clearing).  A producer waits for its block's count before loading q.
+  // CTA adds its rows to the block's counter, (fuse_tag << 16) | rows (the
+  // host clears the counters before the launch, and a counter holding
+  // another launch's tag counts as 0).  A producer waits for its block's
+  // count before loading q.
   const uint16_t *x;
   int64_t ldx;
   int8_t *q_w;
@@ -112,8 +114,6 @@ struct GemmParams {
   unsigned long long *row_ready;   // cdiv(M, 128) counters
   unsigned long long fuse_tag;     // 1 .. 2^48 - 1
 };
-
-constexpr unsigned long long kSplitEpochMask = (1ull << 56) - 1;
 
 // One epilogue warp slice of a 256 x 256 pair tile: 32 rows x 128 columns.
 constexpr int kSlotInts = 32 * 128;
