@@ -3,7 +3,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload qkv|ffn_up|ffn_down|adaln_m1|adaln_m2]
-                    [--no-extras] [--no-e2e] [--no-cpu-baseline] [--cpu-budget S]
+                    [--no-extras] [--no-sweep] [--no-e2e] [--no-cpu-baseline]
+                    [--cpu-budget S]
 
 A step is one whole layer call on one batch: per-token quantization of the
 bf16 activations, the int8 tensor-core GEMM and the fused dequantization
@@ -22,12 +23,18 @@ Beside the headline line's own figures (roofline of the dominant kernel,
 end-to-end time from pinned host buffers, CPU oracle baseline, clocks sampled
 during the timed region), `components` reports the other workloads: the
 AdaLN GEMV at M = 1 and 2, the FFN layers alone and back to back, one DiT
-block's linears at CFG batch 2, the small-M regime, packed-weight loading
-and the W8A16 variant.
+block's linears at CFG batch 2, the small-M regime, the M sweep over the
+block's four linear shapes (32 points), packed-weight loading and the W8A16
+variant.  The roofline's denominator is measured in the same run: the
+tcgen05 kind::i8 instruction issued back to back on every CTA pair with no
+memory traffic; torch._int_mm at 8192^3 is reported beside it as the
+library's rate.
 
 Multi-GPU: the layer shards into independent problems, so N ranks run N
 replicas with no collective on the data path (weak scaling); `value` is the
-sum over ranks.  Launched under torchrun, one rank per GPU.
+sum over ranks.  One rank per GPU: `--gpus N` started without a launcher
+re-executes itself under torchrun with N ranks; under torchrun it reads
+RANK / LOCAL_RANK / WORLD_SIZE.  At N > 1 the extra components are skipped.
 
 --impl reference times the CPU oracle (plain C, OpenMP) on rank 0 on a
 bounded row sample of the same workload; the other ranks exit without work.
@@ -192,16 +199,23 @@ def kernel_source_hash(kernel_tag: str = "") -> str:
 class Layer:
     """One workload's device buffers, rotated over several independent sets."""
 
-    def __init__(self, case: synth.LayerCase, device, with_ws=True):
+    def __init__(self, case: synth.LayerCase, device, with_ws=True, x_bits=None, weights=None):
+        """weights: (Wq, s_w) already quantized on the device, to share one
+        weight between several layers of the same (K, N); x_bits: the host
+        activations when the caller has generated them already."""
         import w8a8_int8_dynamic_token_b200 as w8a8
         self.w8a8 = w8a8
         self.case = case
         M, K, N = case.M, case.K, case.N
-        x_bits, w_bits, b_bits = case.x(), case.w(), case.b()
+        x_bits = case.x() if x_bits is None else x_bits
+        b_bits = case.b()
         x0 = bf16_dev(x_bits, device)
-        W = bf16_dev(w_bits, device)
-        Wq, s_w = w8a8.quantize_weights(W)          # load-time weight quantization
-        del W
+        if weights is None:
+            W = bf16_dev(case.w(), device)
+            Wq, s_w = w8a8.quantize_weights(W)      # load-time weight quantization
+            del W
+        else:
+            Wq, s_w = weights
         b0 = bf16_dev(b_bits, device) if b_bits is not None else None
         self.ws_bytes = w8a8.workspace_size(M, N, K) if with_ws else 0
         per_set = 2 * M * K + N * K + 6 * N + 2 * M * N + self.ws_bytes
@@ -393,18 +407,100 @@ def single_launch_us(fn, reps: int = 20) -> float:
     return statistics.median(times)
 
 
+METRIC = "W8A8 linear int8 TOPS & % of tensor peak (quant+GEMM); M=1 GEMV HBM GB/s"
+DTYPE = "int8 (int32 accumulate, fp32 epilogue, bf16 in/out)"
+L2_NOTE = "inputs rotate over independent buffer sets totalling > 2x the 126 MB L2"
+
+
+def workload_config(case: synth.LayerCase) -> dict:
+    """The `config` of the JSON line: the workload alone, identical for both
+    arms (no rank count, device or kernel choice in it)."""
+    return {"workload": f"{case.name}: x bf16 [{case.M},{case.K}] ({case.x_kind}) @ Wq int8 "
+                        f"[{case.N},{case.K}] + bias -> y bf16",
+            "M": case.M, "K": case.K, "N": case.N, "seed": case.seed,
+            "parallelism": "replicas (one independent layer call per GPU, no collective)",
+            "l2": L2_NOTE}
+
+
+def init_dist(world: int, local: int):
+    """One process per GPU over NCCL, for the barrier around the timed region
+    and the max-over-ranks reduction of the time."""
+    if world <= 1:
+        return None
+    import torch.distributed as tdist
+    from datetime import timedelta
+    tdist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                             device_id=torch.device("cuda", local))
+    return tdist
+
+
+def build_line(args, m: dict, world: int) -> dict:
+    """The JSON line of our arm from the measurements `m` (times already the
+    max over ranks).  `value` is the whole job's rate: the operations of all
+    `world` replicas over the slowest rank's time."""
+    value = job_rate(m["ops_per_step"], args.steps, m["seconds"], world) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": m["warmup"],
+        "ms_per_step": round(m["seconds"] / args.steps * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": DTYPE, "data": "synthetic", "impl": "ours",
+        "config": m["config"],
+        "roofline": m.get("roofline"),
+        "cpu_baseline": m.get("cpu_baseline"),
+        "e2e": m.get("e2e"),
+        "gpu_launches": m["launches_per_step"] * args.steps,
+        "clocks": m.get("clocks"),
+        "run": m.get("run"),
+        "extras": m.get("extras"),
+        "components": m.get("components", {}),
+    }
+    return line
+
+
+def measure_i8_peak(dev, dist=None, iters: int = 10000, reps: int = 5) -> dict:
+    """The device's dense int8 tensor-core rate, measured now: every CTA pair
+    issues the GEMM's own tcgen05 kind::i8 instruction (M = N = 256, K = 32)
+    from shared-memory operands, no global traffic, ~2.5 ms per launch."""
+    import w8a8_int8_dynamic_token_b200 as w8a8
+    B = w8a8.binding
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    pairs = sms // 2
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    t = timed(lambda: B.bench_mma_i8_peak(iters, pairs), reps, 2, dist, sampler) / reps
+    status = w8a8.last_device_error()
+    if status != 0:
+        raise RuntimeError(f"peak loop: {w8a8.status_string(status)}")
+    ops = pairs * iters * B.PEAK_OPS_PER_PAIR_ITERATION
+    clk = sampler.summary()
+    res = {"tops": round(ops / t / 1e12, 1), "us_per_launch": round(t * 1e6, 1),
+           "pairs": pairs, "sm_mhz": clk.get("sm_mhz"), "clock_reasons": clk.get("reasons")}
+    if clk.get("sm_mhz"):
+        res["ops_per_clk_per_sm"] = round(ops / t / (clk["sm_mhz"] * 1e6) / (2 * pairs), 1)
+    return res
+
+
+def measure_int_mm(dev, dist=None, n: int = 8192, reps: int = 20) -> dict:
+    """Library reference point: torch._int_mm (cuBLASLt int8 GEMM) at n^3,
+    operands resident, the same int8 operation count convention."""
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev).t()
+    try:
+        torch._int_mm(a, b)
+    except Exception as e:  # not available in this build: say so
+        return {"error": str(e)[:200]}
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    t = timed(lambda: torch._int_mm(a, b), reps, 3, dist, sampler) / reps
+    del a, b
+    torch.cuda.empty_cache()
+    return {"tops": round(2.0 * n ** 3 / t / 1e12, 1), "us": round(t * 1e6, 1), "n": n,
+            "sm_mhz": sampler.summary().get("sm_mhz")}
+
+
 def run_ours(args):
     rank, world, local = env_rank()
-    dist = None
-    if world > 1:
-        import torch.distributed as tdist
-        from datetime import timedelta
-        torch.cuda.set_device(local)
-        tdist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                 device_id=torch.device("cuda", local))
-        dist = tdist
-    else:
-        torch.cuda.set_device(0)
+    torch.cuda.set_device(local if world > 1 else 0)
+    dist = init_dist(world, local)
     dev = torch.device("cuda", torch.cuda.current_device())
     import w8a8_int8_dynamic_token_b200 as w8a8
     w8a8.lib()
@@ -413,6 +509,7 @@ def run_ours(args):
     M, K, N = case.M, case.K, case.N
     ops = 2.0 * M * N * K
     warmup = max(3, args.warmup)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     layer = Layer(case, dev)
     gemv = layer.variant == "gemv"
@@ -422,7 +519,6 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device error after the timed region: {w8a8.status_string(status)}")
     sec_per_step = t / args.steps
-    value = job_rate(ops, args.steps, t, world) / 1e12
 
     # the same layer with the host launch cost removed (CUDA graph of the steps)
     layer.i = 0
@@ -443,28 +539,40 @@ def run_ours(args):
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                     "traffic": traffic, "kernel": "gemv_i8 (fused quant prologue)",
-                    "peak_basis": f"{peaks['source']} HBM copy bandwidth",
+                    "peak_basis": f"{peaks['source']} HBM copy bandwidth (MEASURED_PEAKS.json)",
                     "algorithmic_bytes_per_launch": algo_bytes,
                     "us_per_launch": round(sec_per_step * 1e6, 2),
                     "timing": "CUDA graph of back-to-back calls"}
     else:
-        int8_peak = peaks["bf16_tflops"] * (NOMINAL_INT8_TOPS / NOMINAL_BF16_TFLOPS)
+        i8 = measure_i8_peak(dev, dist)
+        int_mm = measure_int_mm(dev, dist) if world == 1 else None
+        derived = peaks["bf16_tflops"] * (NOMINAL_INT8_TOPS / NOMINAL_BF16_TFLOPS)
         achieved = ops / tg / 1e12
         traffic, _ = profile_traffic(f"gemm_i8_tcgen05_{case.name}")
-        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_peak, 1),
-                    "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4),
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": i8["tops"],
+                    "unit": "TFLOP/s", "frac": round(achieved / i8["tops"], 4),
                     "traffic": traffic,
                     "kernel": f"gemm_i8_tcgen05 ({layer.variant})",
-                    "peak_basis": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
-                                  f"nominal int8/bf16 ratio 2 (int8 ops counted as TOPS)",
+                    "peak_basis": ("measured in this run: the tcgen05 kind::i8 M=256 N=256 K=32 "
+                                   f"issue loop on all {i8['pairs']} CTA pairs, no memory traffic "
+                                   "(int8 ops counted as TOPS)"),
+                    "peak_measured_i8": i8,
+                    "peak_bf16_x2": round(derived, 1),
+                    "frac_of_peak_bf16_x2": round(achieved / derived, 4),
+                    "peak_bf16_x2_basis": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TFLOP/s "
+                                          "(MEASURED_PEAKS.json) x nominal int8/bf16 ratio 2",
                     "frac_of_nominal_4500": round(achieved / NOMINAL_INT8_TOPS, 4),
                     "us_per_launch": round(tg * 1e6, 2),
                     "sm_mhz_during_gemm": gclk.get("sm_mhz")}
-        if gclk.get("sm_mhz"):
-            # dense int8 tcgen05 rate: 16384 ops per SM per clock
-            clock_peak = 148 * 16384 * gclk["sm_mhz"] * 1e6 / 1e12
-            roofline["frac_of_clock_peak"] = round(achieved / clock_peak, 4)
-            roofline["clock_peak_tops"] = round(clock_peak, 1)
+        if int_mm is not None:
+            roofline["torch_int_mm_8192"] = int_mm
+            if int_mm.get("tops"):
+                roofline["frac_of_torch_int_mm_8192"] = round(achieved / int_mm["tops"], 4)
+        if gclk.get("sm_mhz") and i8.get("ops_per_clk_per_sm"):
+            # the measured per-clock rate at the clock the GEMM itself ran at
+            clock_peak = sms * i8["ops_per_clk_per_sm"] * gclk["sm_mhz"] * 1e6 / 1e12
+            roofline["frac_of_peak_at_gemm_clock"] = round(achieved / clock_peak, 4)
+            roofline["peak_at_gemm_clock_tops"] = round(clock_peak, 1)
     quant_bytes = 3 * M * K + 4 * M
     layer.i = 0
     t_single = single_launch_us(layer.step)
@@ -479,7 +587,6 @@ def run_ours(args):
         "quant_gbs": round(quant_bytes / tq / 1e9, 1),
         "quant_frac_hbm": round(quant_bytes / tq / 1e9 / peaks["hbm_gbs"], 4),
     }
-    gpu_launches = layer.launches_per_step * args.steps
 
     e2e = None
     if not args.no_e2e:
@@ -488,12 +595,14 @@ def run_ours(args):
         e2e = {"value": round(job_rate(ops, esteps, te, world) / 1e12, 3), "unit": "TOPS",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(te / esteps * 1e3, 3)}
+    launches = layer.launches_per_step
     del layer
     torch.cuda.empty_cache()
 
     components = {}
-    if not args.no_extras:
-        components = extra_components(args, dev, dist, peaks, world)
+    if not args.no_extras and world == 1:
+        components = extra_components(args, dev, dist, peaks, world,
+                                      roofline.get("peak") if not gemv else None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -501,29 +610,13 @@ def run_ours(args):
 
     if dist is not None:
         dist.barrier()
+    m = {"seconds": t, "ops_per_step": ops, "warmup": warmup, "config": workload_config(case),
+         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "launches_per_step": launches,
+         "clocks": sampler.summary(), "extras": extras, "components": components,
+         "run": {"gpu": torch.cuda.get_device_name(dev), "sms": sms,
+                 "kernel_variant": layer_variant_name(case), "ranks": world}}
     if rank == 0:
-        line = {
-            "metric": "W8A8 linear int8 TOPS & % of tensor peak (quant+GEMM); M=1 GEMV HBM GB/s",
-            "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": warmup, "ms_per_step": round(sec_per_step * 1e3, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8 (int32 accumulate, fp32 epilogue, bf16 in/out)", "data": "synthetic",
-            "impl": "ours",
-            "config": {"workload": f"{case.name}: x bf16 [{M},{K}] ({case.x_kind}) @ Wq int8 [{N},{K}] + bias -> y bf16",
-                       "M": M, "K": K, "N": N, "seed": case.seed,
-                       "gpu": torch.cuda.get_device_name(dev),
-                       "parallelism": f"replicas x{world}",
-                       "l2": f"inputs rotate over independent buffer sets totalling > 2x the 126 MB L2",
-                       "kernel_variant": layer_variant_name(case)},
-            "roofline": roofline,
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": gpu_launches,
-            "clocks": sampler.summary(),
-            "extras": extras,
-            "components": components,
-        }
-        print(json.dumps(line), flush=True)
+        print(json.dumps(build_line(args, m, world)), flush=True)
     if dist is not None:
         dist.destroy_process_group()
 
@@ -533,9 +626,11 @@ def layer_variant_name(case):
     return w8a8.select(case.M, case.N, case.K)["variant_name"]
 
 
-def extra_components(args, dev, dist, peaks, world):
+def extra_components(args, dev, dist, peaks, world, i8_peak=None):
     """The other workloads of the same metric: the M = 1 / 2 AdaLN GEMV (HBM
-    GB/s), and the FFN up/down pair, each layer alone and back to back."""
+    GB/s), the FFN up/down pair, each layer alone and back to back, one DiT
+    block, the small-M regime, the M sweep over the block's linear shapes,
+    packed-weight loading and the W8A16 variant."""
     out = {}
     steps = max(20, min(args.steps, 200))
     for case in (synth.ADALN_M1, synth.ADALN_M2):
@@ -576,6 +671,8 @@ def extra_components(args, dev, dist, peaks, world):
         torch.cuda.empty_cache()
         out["dit_block"] = dit_block_component(dev, dist, max(10, steps // 4))
         out["small_m"] = small_m_component(dev, dist, peaks, steps)
+        if not args.no_sweep:
+            out["sweep"] = sweep_component(dev, dist, peaks, i8_peak)
         out["unpack_int32_weights"] = unpack_component(dev, dist, peaks, steps)
         out["w8a16_qkv"] = w8a16_component(dev, dist, peaks, steps)
     return out
@@ -608,6 +705,64 @@ def w8a16_component(dev, dist, peaks, steps):
     return {"us": round(t * 1e6, 2), "TFLOPS": round(tflops, 1),
             "frac_of_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
             "peak_basis": "measured bf16 burst (MEASURED_PEAKS.json)"}
+
+
+def sweep_component(dev, dist, peaks, i8_peak, oracle_rows: int = 4):
+    """The M sweep over one DiT block's linear shapes: M in {1, 16, 17, 256,
+    1024, 4352, 8704, 16384} x (K, N) in {(3072, 9216), (3072, 3072),
+    (3072, 12288), (12288, 3072)}, seed 0 (seeds 1-3 are parity cases).  Per
+    point: the whole layer (quantization included) in a CUDA graph of
+    back-to-back calls with inputs rotated over > 2x L2, its TOPS, the
+    algorithmic GB/s, and the fraction of the attainable rate
+    min(peak_i8, AI * HBM) with AI = 2MNK / (2MK + NK + 6N + 2MN); and the
+    oracle's rate on a few rows of the same layer (plain C, all host cores)."""
+    import oracle
+    points = []
+    bw = peaks["hbm_gbs"] * 1e9
+    for K, N in synth.SWEEP_KN:
+        kind = "gelu" if K == 12288 else "studentt"
+        w_bits = synth.make_w(N, K, 0)
+        weights = quantized_weights(w_bits, dev)
+        wq_h, sw_h = oracle.quantize_weights(w_bits)
+        for M in synth.SWEEP_M:
+            case = synth.LayerCase(f"sweep_m{M}_k{K}_n{N}_s0", M, K, N, kind, 0)
+            x_bits = case.x()
+            L = Layer(case, dev, x_bits=x_bits, weights=weights)
+            ops = 2.0 * M * N * K
+            steps = int(min(200, max(10, 2e-2 / max(ops / 3e15, 2e-6))))   # ~20 ms of work
+            t = timed(L.step, steps, 3, dist, graph=True) / steps
+            algo = 2 * M * K + N * K + 6 * N + 2 * M * N
+            ai = ops / algo
+            attain = min(i8_peak * 1e12 if i8_peak else NOMINAL_INT8_TOPS * 1e12, ai * bw)
+            rows = min(M, oracle_rows)
+            t0 = time.perf_counter()
+            oracle.linear(x_bits[:rows], wq_h, sw_h, case.b())
+            t_or = time.perf_counter() - t0
+            points.append({"M": M, "K": K, "N": N, "variant": L.variant, "us": round(t * 1e6, 2),
+                           "TOPS": round(ops / t / 1e12, 1), "GBs": round(algo / t / 1e9, 1),
+                           "bound": "tensor" if ai * bw > attain * 0.999 else "hbm",
+                           "frac_of_attainable": round(ops / t / attain, 4),
+                           "frac_of_nominal_4500": round(ops / t / 1e12 / NOMINAL_INT8_TOPS, 4),
+                           "oracle_TOPS": round(2.0 * rows * N * K / t_or / 1e12, 5),
+                           "oracle_rows": rows})
+            del L
+            torch.cuda.empty_cache()
+        del weights
+        torch.cuda.empty_cache()
+    return {"points": points,
+            "attainable": "min(measured int8 peak of this run, AI x measured HBM GB/s)",
+            "timing": "CUDA graph of back-to-back layer calls (quantization + GEMM or the GEMV), "
+                      "inputs rotated over > 2x L2; seed 0",
+            "oracle": f"CPU oracle on the first {oracle_rows} rows of each layer, all outputs"}
+
+
+def quantized_weights(w_bits, dev):
+    """Quantize a host bf16 weight once on the device, for several layers."""
+    import w8a8_int8_dynamic_token_b200 as w8a8
+    W = bf16_dev(w_bits, dev)
+    Wq, s_w = w8a8.quantize_weights(W)
+    del W
+    return Wq, s_w
 
 
 def small_m_component(dev, dist, peaks, steps):
@@ -718,20 +873,40 @@ def run_reference(args):
     sample = (f"{rows} of {M} rows of the {case.name} layer per step (all {N} outputs per row): "
               f"per-token quant + exact int32 GEMM + fp32 epilogue, plain C with OpenMP")
     line = {
-        "metric": "W8A8 linear int8 TOPS & % of tensor peak (quant+GEMM); M=1 GEMV HBM GB/s",
+        "metric": METRIC,
         "value": round(value, 6), "unit": "TOPS", "n_gpus": world, "steps": len(times),
         "warmup": max(3, args.warmup), "ms_per_step": round(t / len(times) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8 (int32 accumulate, fp32 epilogue, bf16 in/out)", "data": "synthetic",
+        "dtype": DTYPE, "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": f"{case.name}: x bf16 [{M},{K}] ({case.x_kind}) @ Wq int8 [{N},{K}] + bias -> y bf16",
-                   "M": M, "K": K, "N": N, "seed": case.seed, "parallelism": "rank 0 only"},
+        "config": workload_config(case),
+        "run": {"ranks": world, "oracle_on": "rank 0 only"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": oracle.threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def launcher_argv(n: int, port: int, argv=None) -> list:
+    """The torchrun command that runs this script as n ranks on this node,
+    one per GPU, rendezvous on 127.0.0.1."""
+    argv = sys.argv[1:] if argv is None else argv
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
+def relaunch_under_torchrun(n: int):
+    """`--gpus N` without a launcher: replace this process by torchrun with N
+    ranks (each rank then sees WORLD_SIZE and runs its replica)."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    sys.stdout.flush()
+    cmd = launcher_argv(n, port)
+    os.execv(cmd[0], cmd)
 
 
 def main():
@@ -745,7 +920,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-sweep", action="store_true")
     args = ap.parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        relaunch_under_torchrun(args.gpus)   # does not return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -83,8 +83,12 @@ typedef enum {
     W8A8_VARIANT_GEMM_BN128 = 2,    /* tcgen05 kind::i8, 128x128 tiles */
     W8A8_VARIANT_GEMM_BN256 = 3,    /* tcgen05 kind::i8, 128x256 tiles */
     W8A8_VARIANT_GEMM_PAIR = 4,     /* tcgen05 kind::i8 on CTA pairs, 256x256 tiles */
-    W8A8_VARIANT_GEMM_BN64 = 5      /* tcgen05 kind::i8, 128x64 tiles (small M: more
+    W8A8_VARIANT_GEMM_BN64 = 5,     /* tcgen05 kind::i8, 128x64 tiles (small M: more
                                        CTAs streaming the weights) */
+    W8A8_VARIANT_GEMV_TC = 6        /* M <= 128: tcgen05 kind::i8 with the weights as
+                                       the MMA's 128-row side and the activation rows
+                                       (padded to 16/32/64/128) as its N side; K split
+                                       among the CTAs of a cluster when tiles are few */
 } w8a8_variant;
 
 /* The selector's decision for one (M, N, K); see w8a8_select. */
@@ -108,6 +112,8 @@ typedef struct {
                               with W8A8_FUSED_ONE_LAUNCH can run the per-token
                               quantization inside the GEMM launch (given the
                               full workspace, outside stream capture); else 0 */
+    int32_t k_split;       /* GEMV_TC: CTAs (one cluster) sharing each 128-row
+                              weight tile along K, 1..8; else 0 */
 } w8a8_plan;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -322,6 +328,18 @@ W8A8_API int w8a8_linear_fused_noalloc(const void *x_bf16, int64_t M, int64_t K,
  * on the order of a second.
  */
 W8A8_API int w8a8_selftest_quant_exhaustive(unsigned long long *counts_dev, w8a8_stream_t stream);
+
+/*
+ * Measurement of the device's int8 tensor-core ceiling, the denominator of
+ * the GEMM's roofline: `pairs` CTA pairs (1 .. SMs / 2) each issue
+ * 4 * iterations tcgen05.mma.cta_group::2.kind::i8 instructions (M = 256,
+ * N = 256, K = 32: the GEMM's own instruction) from operands held in shared
+ * memory, with no global-memory traffic.  The launch performs
+ * pairs * iterations * 16,777,216 int8 operations; the caller times it
+ * (CUDA events on `stream`).  iterations: 1 .. 500000 (a fraction of a
+ * second), else W8A8_ERR_INVALID_ARG.  Asynchronous; nothing is allocated.
+ */
+W8A8_API int w8a8_bench_mma_i8_peak(int64_t iterations, int32_t pairs, w8a8_stream_t stream);
 
 /*
  * Test support: the launch tag that the next call using arrival counters

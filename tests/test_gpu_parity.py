@@ -51,6 +51,8 @@ def _quant_check(x_bits, q_dev, s_dev):
 @pytest.mark.parametrize("M,K,kind", [
     (64, 256, "outlier20"), (300, 3072, "studentt"), (17, 12288, "gelu"), (5, 16, "normal"),
     (1000, 4096, "normal"), (3, 133120, "normal"), (7, 2064, "studentt"), (33, 24576, "gelu"),
+    # more rows than one pass of every warp's slots: the slot rings are refilled
+    (20000, 256, "normal"), (9000, 4096, "studentt"), (2000, 12288, "gelu"), (4353, 3072, "studentt"),
 ])
 def test_quant_act_bitexact(M, K, kind):
     x = synth.make_x(M, K, kind, seed=M)
@@ -92,6 +94,18 @@ def test_quant_edge_rows(K):
     q_ref, s_ref = _quant_check(x, q, s)
     assert s_ref[0] == 0 and not q_ref[0].any()
     assert q_ref[4].min() == 127                                # all-equal subnormal row
+
+
+def test_int8_peak_loop_runs_clean():
+    """The tensor-core ceiling measurement: every CTA pair issues MMAs from
+    shared memory; the launch must complete with no device error."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for pairs, iters in ((1, 10), (sms // 2, 1000)):
+        B.bench_mma_i8_peak(iters, pairs)
+    torch.cuda.synchronize()
+    assert w8a8.last_device_error() == B.W8A8_OK
+    with pytest.raises(w8a8.W8A8Error):
+        B.bench_mma_i8_peak(500001, 1)          # beyond the bounded length
 
 
 def test_division_free_quant_step_exhaustive():
@@ -211,6 +225,53 @@ def test_gemv_fused_and_unfused(M, N, K):
         assert check_y(bits_of(yy), ref["y"], ref["y32"], "gemv") == 0
 
 
+# (M, N, K): activation rows padded to 16 / 32 / 64 / 128; one tile
+# (128 x 256, K shared by up to 8 CTAs), ragged N (1032), K not a multiple of
+# 128 (2064), the AdaLN shape (144 tiles, no split), the QKV weight (72 tiles,
+# K in two halves) and N = 3072 (24 tiles, K in six parts).
+GEMV_TC_CASES = [(1, 128, 256), (2, 18432, 3072), (5, 1032, 2064), (16, 9216, 3072),
+                 (17, 3072, 3072), (31, 3072, 12288), (64, 264, 3072), (100, 9216, 3072),
+                 (128, 1032, 12288), (3, 128, 16)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMV_TC_CASES)
+def test_gemv_tc_int32_exact_and_y(M, N, K):
+    """The tensor-core small-M variant (weights on the MMA's 128-row side,
+    K split among the CTAs of a cluster, partial sums added in distributed
+    shared memory): raw int32 equal to the oracle, y bit-equal."""
+    plan = w8a8.select(M, N, K, variant=B.VARIANT_GEMV_TC)
+    assert plan["k_split"] >= 1 and plan["grid"] == plan["num_tiles"] * plan["k_split"]
+    x, w, b = synth.make_x(M, K, "studentt", M + 3), synth.make_w(N, K, M + 3), synth.make_bias(N, M + 3)
+    wq_ref, sw_ref = oracle.quantize_weights(w)
+    ref = oracle.linear(x, wq_ref, sw_ref, b)
+    args = (torch.from_numpy(ref["q"]).cuda(), torch.from_numpy(ref["s_a"]).cuda(),
+            torch.from_numpy(wq_ref).cuda(), torch.from_numpy(sw_ref).cuda())
+    acc = w8a8.linear(*args, acc_debug=True, variant=B.VARIANT_GEMV_TC)
+    y = w8a8.linear(*args, to_dev(b), variant=B.VARIANT_GEMV_TC)
+    y_nobias = w8a8.linear(*args, variant=B.VARIANT_GEMV_TC)
+    torch.cuda.synchronize()
+    assert np.array_equal(acc.cpu().numpy(), ref["acc"])
+    assert check_y(bits_of(y), ref["y"], ref["y32"], "gemv_tc") == 0
+    y32n, yn = oracle.epilogue(ref["acc"], ref["s_a"], sw_ref, None)
+    assert check_y(bits_of(y_nobias), yn, y32n, "gemv_tc no bias") == 0
+
+
+def test_gemv_tc_extremes_at_max_k():
+    K = 133120
+    q = np.full((3, K), 127, np.int8)
+    q[1] = -127
+    q[2, ::2] = -127
+    wq = np.full((136, K), 127, np.int8)
+    wq[5, ::2] = -127
+    acc = w8a8.linear(torch.from_numpy(q).cuda(), torch.ones(3, device="cuda"),
+                      torch.from_numpy(wq).cuda(), torch.ones(136, device="cuda"),
+                      acc_debug=True, variant=B.VARIANT_GEMV_TC)
+    torch.cuda.synchronize()
+    ref = oracle.gemm_i32(q, wq)
+    assert ref[0, 0] == 127 * 127 * K and ref[1, 0] == -127 * 127 * K
+    assert np.array_equal(acc.cpu().numpy(), ref)
+
+
 def test_gemm_variant_at_tiny_m_matches_gemv():
     M, N, K = 3, 264, 512
     x, w, b = synth.make_x(M, K, "normal", 5), synth.make_w(N, K, 5), synth.make_bias(N, 5)
@@ -218,7 +279,8 @@ def test_gemm_variant_at_tiny_m_matches_gemv():
     ref = oracle.linear(x, wq_ref, sw_ref, b)
     args = (torch.from_numpy(ref["q"]).cuda(), torch.from_numpy(ref["s_a"]).cuda(),
             torch.from_numpy(wq_ref).cuda(), torch.from_numpy(sw_ref).cuda(), to_dev(b))
-    for v in (B.VARIANT_GEMV, B.VARIANT_GEMM_BN128, B.VARIANT_GEMM_BN256, B.VARIANT_GEMM_PAIR):
+    for v in (B.VARIANT_GEMV, B.VARIANT_GEMM_BN128, B.VARIANT_GEMM_BN256, B.VARIANT_GEMM_PAIR,
+              B.VARIANT_GEMV_TC):
         y = w8a8.linear(*args, variant=v)
         torch.cuda.synchronize()
         assert check_y(bits_of(y), ref["y"], ref["y32"], f"variant {v}") == 0

@@ -8,7 +8,7 @@ dequantization/bias epilogue producing bf16.  The kernels live in
 """
 from .binding import (  # noqa: F401
     LIB_PATH, VARIANT_AUTO, VARIANT_GEMM_BN64, VARIANT_GEMM_BN128, VARIANT_GEMM_BN256,
-    VARIANT_GEMM_PAIR, VARIANT_GEMV,
+    VARIANT_GEMM_PAIR, VARIANT_GEMV, VARIANT_GEMV_TC,
     W8A8Error, last_device_error, lib, linear, linear_fused, linear_fused_host, quant_act,
     quantize_weights, select, selftest_bounded_wait, status_string, unpack_int32_weights, version,
     w8a16_linear, workspace_size,

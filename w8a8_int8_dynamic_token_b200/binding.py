@@ -39,8 +39,9 @@ VARIANT_GEMM_BN128 = 2
 VARIANT_GEMM_BN256 = 3
 VARIANT_GEMM_PAIR = 4
 VARIANT_GEMM_BN64 = 5
+VARIANT_GEMV_TC = 6
 VARIANT_NAMES = {0: "auto", 1: "gemv", 2: "gemm_bn128", 3: "gemm_bn256", 4: "gemm_pair",
-                 5: "gemm_bn64"}
+                 5: "gemm_bn64", 6: "gemv_tc"}
 
 
 class W8A8Error(RuntimeError):
@@ -54,7 +55,8 @@ class Plan(ctypes.Structure):
                 ("tile_n", ctypes.c_int32), ("num_tiles", ctypes.c_int32),
                 ("grid", ctypes.c_int32), ("waves_x100", ctypes.c_int32),
                 ("split_tiles", ctypes.c_int32), ("split_kblocks_per_pair", ctypes.c_int32),
-                ("tail_tiles_nsplit", ctypes.c_int32), ("quant_in_gemm_launch", ctypes.c_int32)]
+                ("tail_tiles_nsplit", ctypes.c_int32), ("quant_in_gemm_launch", ctypes.c_int32),
+                ("k_split", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {f: getattr(self, f) for f, _ in self._fields_}
@@ -89,6 +91,7 @@ _SIGNATURES = {
     "w8a8_selftest_bounded_wait": ([_i64, _vp], _int),
     "w8a8_selftest_quant_exhaustive": ([_vp, _vp], _int),
     "w8a8_debug_peek_tag": ([ctypes.POINTER(ctypes.c_uint64)], _int),
+    "w8a8_bench_mma_i8_peak": ([_i64, _i32, _vp], _int),
 }
 
 
@@ -466,6 +469,16 @@ def selftest_quant_exhaustive(stream=None) -> tuple[int, int]:
     torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
     c = counts.cpu().tolist()
     return int(c[0]), int(c[1])
+
+
+PEAK_OPS_PER_PAIR_ITERATION = 4 * 2 * 256 * 256 * 32
+
+
+def bench_mma_i8_peak(iterations: int, pairs: int, stream=None) -> None:
+    """Enqueue the int8 tensor-core peak loop (pairs * iterations *
+    PEAK_OPS_PER_PAIR_ITERATION operations); time it with CUDA events."""
+    _check(lib().w8a8_bench_mma_i8_peak(int(iterations), int(pairs), _stream(stream)),
+           "w8a8_bench_mma_i8_peak")
 
 
 def debug_peek_tag() -> int:

@@ -17,9 +17,11 @@
 #include "w8a8_gemm.cuh"
 #include "w8a8_gemv.cuh"
 #include "w8a8_pack.cuh"
+#include "w8a8_peak.cuh"
 #include "w8a16_gemm.cuh"
 #include "w8a8_ptx.cuh"
 #include "w8a8_quant.cuh"
+#include "w8a8_swapab.cuh"
 
 namespace w8a8 {
 
@@ -113,6 +115,20 @@ inline bool gemv_fits(int64_t M, int64_t K, int max_smem) {
 // there (launch, pipeline fill and epilogue bound); they cross at M = 5-6.
 constexpr int64_t kGemvAutoMaxM = 4;
 
+// The tensor-core small-M variant serves up to this many activation rows.
+constexpr int64_t kSwapMaxM = 128;
+
+inline int swap_mpad(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
+
+inline int swap_max_split(int mpad) {
+  switch (mpad) {
+    case 16: return SwapLayout<16>::kMaxSplit;
+    case 32: return SwapLayout<32>::kMaxSplit;
+    case 64: return SwapLayout<64>::kMaxSplit;
+    default: return SwapLayout<128>::kMaxSplit;
+  }
+}
+
 int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int max_smem,
                 w8a8_plan *plan) {
   if (sms < 1) return W8A8_ERR_INVALID_ARG;
@@ -149,6 +165,25 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
   }
   std::memset(plan, 0, sizeof(*plan));
   plan->variant = v;
+  if (v == W8A8_VARIANT_GEMV_TC) {
+    if (M > kSwapMaxM) return W8A8_ERR_UNSUPPORTED_SHAPE;
+    const int mpad = swap_mpad(M);
+    const int64_t tiles = cdiv(N, kBM);
+    const int64_t kb = cdiv(K, kBK);
+    // K shared among the CTAs of a cluster until the tiles fill the SMs
+    int64_t split = sms / tiles;
+    if (split > swap_max_split(mpad)) split = swap_max_split(mpad);
+    if (split > kb) split = kb;
+    if (split < 1) split = 1;
+    if (tiles * split > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
+    plan->tile_m = kBM;
+    plan->tile_n = mpad;
+    plan->num_tiles = static_cast<int32_t>(tiles);
+    plan->k_split = static_cast<int32_t>(split);
+    plan->grid = static_cast<int32_t>(tiles * split);
+    plan->waves_x100 = static_cast<int32_t>(cdiv(100 * tiles * split, sms));
+    return W8A8_OK;
+  }
   if (v == W8A8_VARIANT_GEMV) {
     if (!gemv_fits(M, K, max_smem)) return W8A8_ERR_UNSUPPORTED_SHAPE;
     const int64_t smem = M * K;
@@ -396,28 +431,41 @@ int encode_bf16_store_map(CUtensorMap *map, const void *base, int64_t rows, int6
 // must call griddepcontrol.wait before touching anything that work produces
 // (the GEMM kernels do, before their first q / s_a read and any store).
 template <typename... KArgs, typename... Args>
-int launch_ex(bool dependent, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-              cudaStream_t stream, Args... args) {
+int launch_cl(bool dependent, unsigned cluster_x, void (*kernel)(KArgs...), dim3 grid, dim3 block,
+              size_t smem, cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cfg.attrs = nullptr;
+  cfg.attrs = attr;
   cfg.numAttrs = 0;
   if (dependent) {
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+    ++cfg.numAttrs;
   }
+  if (cluster_x > 1) {  // a cluster of cluster_x CTAs along x (no multicast loads)
+    attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+    attr[cfg.numAttrs].val.clusterDim.x = cluster_x;
+    attr[cfg.numAttrs].val.clusterDim.y = 1;
+    attr[cfg.numAttrs].val.clusterDim.z = 1;
+    ++cfg.numAttrs;
+  }
+  if (cfg.numAttrs == 0) cfg.attrs = nullptr;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return W8A8_ERR_CUDA;
   }
   return W8A8_OK;
+}
+
+template <typename... KArgs, typename... Args>
+int launch_ex(bool dependent, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+              cudaStream_t stream, Args... args) {
+  return launch_cl(dependent, 1u, kernel, grid, block, smem, stream, args...);
 }
 
 template <typename... KArgs, typename... Args>
@@ -449,10 +497,38 @@ int ensure_smem_limit(int bytes) {
   return W8A8_OK;
 }
 
+// Warps per CTA and row slots per warp of quant_rows_bulk_kernel for rows of
+// K elements: as many warps as fit two slots each in the slot storage (16, 8
+// or 4), then as many slots (up to 4) as fit.
+void quant_bulk_shape(int64_t K, int *warps, int *slots) {
+  const int64_t row_bytes = 2 * K;
+  int w = kQuantBulkMaxWarps;
+  while (w > 4 && w * 2 * row_bytes > kQuantBulkSmem) w /= 2;
+  int64_t sl = kQuantBulkSmem / (w * row_bytes);
+  if (sl > kQuantBulkMaxSlots) sl = kQuantBulkMaxSlots;
+  *warps = w;
+  *slots = static_cast<int>(sl);
+}
+
 int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q, float *s,
                  cudaStream_t stream) {
   const uint16_t *xp = static_cast<const uint16_t *>(x);
   if (rows > INT32_MAX / 2) return W8A8_ERR_UNSUPPORTED_SHAPE;
+  if (K <= kQuantBulkMaxK) {
+    const DeviceInfo *d = nullptr;
+    int st = query_device(&d);
+    if (st != W8A8_OK) return st;
+    int warps = 0, slots = 0;
+    quant_bulk_shape(K, &warps, &slots);
+    const int smem = warps * slots * static_cast<int>(2 * K);
+    st = ensure_smem_limit<quant_rows_bulk_kernel>(kQuantBulkSmem);
+    if (st != W8A8_OK) return st;
+    int64_t grid = cdiv(rows, warps);
+    if (grid > d->sms) grid = d->sms;
+    return launch_ex(true, quant_rows_bulk_kernel, dim3(static_cast<unsigned>(grid)),
+                     dim3(warps * 32), static_cast<size_t>(smem), stream, xp,
+                     static_cast<int>(rows), static_cast<int>(K), ldx, q, s, slots);
+  }
   // G threads per row (32 .. 256), each holding V <= kQuantMaxV vectors of
   // 8 bf16 in registers; longer rows take the two-pass kernel.
   const int64_t nvec = K / 8;
@@ -612,6 +688,47 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
                    mbt, my, p);
 }
 
+template <int MPAD, bool RAW>
+int launch_swapab_t(const w8a8_plan &plan, const int8_t *q, const float *s_a, int64_t M, int64_t K,
+                    const int8_t *wq, const float *s_w, const void *bias, int64_t N, void *y,
+                    int64_t ldy, int32_t *acc, cudaStream_t stream) {
+  using L = SwapLayout<MPAD>;
+  CUtensorMap mw, mq;
+  int st = encode_i8_map(&mw, wq, N, K, kBM);
+  if (st != W8A8_OK) return st;
+  st = encode_i8_map(&mq, q, M, K, MPAD);
+  if (st != W8A8_OK) return st;
+  SwapParams p;
+  p.M = static_cast<int32_t>(M);
+  p.N = static_cast<int32_t>(N);
+  p.K = static_cast<int32_t>(K);
+  p.k_blocks = static_cast<int32_t>(cdiv(K, kBK));
+  p.split = plan.k_split;
+  p.s_a = s_a;
+  p.s_w = s_w;
+  p.bias = static_cast<const uint16_t *>(bias);
+  p.y = static_cast<uint16_t *>(y);
+  p.ldy = ldy;
+  p.acc_out = acc;
+  constexpr auto kernel = gemm_i8_swapab_kernel<MPAD, RAW>;
+  st = ensure_smem_limit<kernel>(L::kSmemBytes);
+  if (st != W8A8_OK) return st;
+  return launch_cl(true, static_cast<unsigned>(plan.k_split), kernel, dim3(plan.grid),
+                   dim3(kSwThreads), L::kSmemBytes, stream, mw, mq, p);
+}
+
+template <bool RAW>
+int launch_swapab(const w8a8_plan &plan, const int8_t *q, const float *s_a, int64_t M, int64_t K,
+                  const int8_t *wq, const float *s_w, const void *bias, int64_t N, void *y,
+                  int64_t ldy, int32_t *acc, cudaStream_t stream) {
+  switch (plan.tile_n) {
+    case 16: return launch_swapab_t<16, RAW>(plan, q, s_a, M, K, wq, s_w, bias, N, y, ldy, acc, stream);
+    case 32: return launch_swapab_t<32, RAW>(plan, q, s_a, M, K, wq, s_w, bias, N, y, ldy, acc, stream);
+    case 64: return launch_swapab_t<64, RAW>(plan, q, s_a, M, K, wq, s_w, bias, N, y, ldy, acc, stream);
+    default: return launch_swapab_t<128, RAW>(plan, q, s_a, M, K, wq, s_w, bias, N, y, ldy, acc, stream);
+  }
+}
+
 template <bool FUSED, bool RAW>
 int launch_gemv_m(const w8a8_plan &plan, const GemvParams &p, cudaStream_t stream) {
   const int smem = p.M * p.K;
@@ -701,6 +818,10 @@ int linear_impl(const int8_t *q, const float *s_a, int64_t M, int64_t K, const i
     p.acc_out = acc;
     return acc ? launch_gemv_m<false, true>(plan, p, stream)
                : launch_gemv_m<false, false>(plan, p, stream);
+  }
+  if (plan.variant == W8A8_VARIANT_GEMV_TC) {
+    return acc ? launch_swapab<true>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc, stream)
+               : launch_swapab<false>(plan, q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc, stream);
   }
   if (plan.variant == W8A8_VARIANT_GEMM_PAIR) {
     const SplitRegion split = split_region(plan, split_ws, split_ws_bytes);
@@ -797,6 +918,16 @@ const char *w8a8_status_string(int status) {
 
 const char *w8a8_version(void) { return "w8a8 1.1 sm_100a"; }
 
+int w8a8_bench_mma_i8_peak(int64_t iterations, int32_t pairs, w8a8_stream_t stream) {
+  if (iterations < 1 || iterations > 500000 || pairs < 1) return W8A8_ERR_INVALID_ARG;
+  const DeviceInfo *d = nullptr;
+  int st = query_device(&d);
+  if (st != W8A8_OK) return st;
+  if (pairs > d->sms / 2) return W8A8_ERR_INVALID_ARG;
+  return launch(mma_i8_peak_kernel, dim3(static_cast<unsigned>(2 * pairs)), dim3(kPeakThreads),
+                kPeakSmemBytes, reinterpret_cast<cudaStream_t>(stream), iterations);
+}
+
 int w8a8_debug_peek_tag(uint64_t *tag) {
   if (!tag) return W8A8_ERR_INVALID_ARG;
   const unsigned long long t = g_tag.load(std::memory_order_relaxed) & ((1ull << 56) - 1);
@@ -885,8 +1016,7 @@ int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K, cons
                    const float *s_w, const void *bias, int64_t N, void *y, int64_t ldy,
                    int32_t *acc_debug, int variant, void *workspace, size_t ws_bytes,
                    w8a8_stream_t stream) {
-  if (variant < W8A8_VARIANT_AUTO || variant > W8A8_VARIANT_GEMM_BN64)
-    return W8A8_ERR_INVALID_ARG;
+  if (variant < W8A8_VARIANT_AUTO || variant > W8A8_VARIANT_GEMV_TC) return W8A8_ERR_INVALID_ARG;
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, acc_debug, variant, workspace,
                      ws_bytes, false, reinterpret_cast<cudaStream_t>(stream));
 }

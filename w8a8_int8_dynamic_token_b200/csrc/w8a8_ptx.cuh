@@ -188,6 +188,18 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_
       : "memory");
 }
 
+// Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from global memory into this CTA's shared memory; the mbarrier
+// receives the byte count.  No multicast.
+__device__ __forceinline__ void bulk_load_g2s(void *dst, const void *src, uint32_t bytes,
+                                              uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // 2-D tiled store of the smem box at (x = inner element, y = row) to global
 // memory; elements outside the tensor are not written.  Tracked as a bulk
 // group of the issuing thread.

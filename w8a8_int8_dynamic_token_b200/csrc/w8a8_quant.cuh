@@ -28,6 +28,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "w8a8_ptx.cuh"
 
 namespace w8a8 {
 
@@ -201,8 +202,95 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const uint16_t *__
   }
 }
 
-// The hot-path kernel: a group of G threads owns one row (G = 32, one warp,
-// whenever the row fits in 12 vectors per lane; K = 3072 gives 12).  Each
+// ---------------------------------------------------------------------------
+// The hot-path kernel for rows of up to kQuantBulkMaxK elements: one CTA per
+// SM, persistent, W warps, each warp owning one row at a time.  Rows reach
+// shared memory by bulk copies (one cp.async.bulk per row), S slots per warp,
+// so each warp has S rows in flight and a CTA W * S * 2K bytes -- the whole
+// CTA's share of a 4352 x 3072 layer is requested at once.  Warp w of CTA c
+// takes rows c * W + w + i * gridDim.x * W, i = 0, 1, ..., so rows complete
+// roughly in order across the GPU.  Per row: max |x| over the slot (bit
+// patterns, warp shuffles), the scale and its reciprocal, then the codes from
+// the slot with the division-free step, 8 bytes per lane per store.  Every
+// slot wait is bounded; on expiry the warp waits for its copies in flight and
+// the kernel returns with the device error word set.
+constexpr int kQuantBulkMaxK = 12288;
+constexpr int kQuantBulkSmem = 196608;   // slot storage per CTA
+constexpr int kQuantBulkMaxWarps = 16;
+constexpr int kQuantBulkMaxSlots = 4;
+
+__global__ void __launch_bounds__(kQuantBulkMaxWarps * 32, 1)
+    quant_rows_bulk_kernel(const uint16_t *__restrict__ x, int rows, int K, int64_t ldx,
+                           int8_t *__restrict__ q, float *__restrict__ s, int slots) {
+  extern __shared__ __align__(128) uint8_t quant_slots[];
+  __shared__ uint64_t bars[kQuantBulkMaxWarps * kQuantBulkMaxSlots];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
+  uint8_t *mine = quant_slots + static_cast<size_t>(warp) * slots * row_bytes;
+  uint64_t *bar = bars + warp * kQuantBulkMaxSlots;
+  const int stride = static_cast<int>(gridDim.x) * warps;
+  const int first = static_cast<int>(blockIdx.x) * warps + warp;
+  const int n_rows = first < rows ? (rows - first + stride - 1) / stride : 0;
+  if (threadIdx.x == 0) abort_flag = 0;
+  if (lane == 0)
+    for (int j = 0; j < slots; ++j) mbar_init(&bar[j], 1);
+  fence_mbarrier_init();
+  __syncthreads();
+  // launched as a programmatic dependent: x may come from the preceding
+  // kernel, and q / s may still be read by it
+  grid_dependency_wait();
+  int issued = 0;
+  if (lane == 0) {
+    for (; issued < slots && issued < n_rows; ++issued) {
+      const int64_t row = first + static_cast<int64_t>(issued) * stride;
+      mbar_arrive_expect_tx(&bar[issued], row_bytes);
+      bulk_load_g2s(mine + issued * row_bytes, x + row * ldx, row_bytes, &bar[issued]);
+    }
+  }
+  grid_dependents_launch();  // the GEMM that follows may start its prologue
+  const int nvec = K >> 3;
+  int i = 0;
+  for (; i < n_rows; ++i) {
+    const int slot = i % slots;
+    int ok = mbar_wait(&bar[slot], static_cast<uint32_t>(i / slots) & 1u, &abort_flag) ? 1 : 0;
+    if (!__all_sync(0xFFFFFFFFu, ok)) break;
+    const int64_t row = first + static_cast<int64_t>(i) * stride;
+    const uint4 *xs = reinterpret_cast<const uint4 *>(mine + slot * row_bytes);
+    float m0 = 0.0f, m1 = 0.0f;
+    int vi = lane;
+    for (; vi + 32 < nvec; vi += 64) {
+      m0 = absmax_vec8(xs[vi], m0);
+      m1 = absmax_vec8(xs[vi + 32], m1);
+    }
+    if (vi < nvec) m0 = absmax_vec8(xs[vi], m0);
+    const float amax = __uint_as_float(warp_max_u32(__float_as_uint(fmaxf(m0, m1)), 32));
+    const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+    const bool fast = quant_fast_ok(sc);
+    const float rc = fast ? __frcp_rn(sc) : 0.0f;
+    if (lane == 0) s[row] = sc;
+    uint2 *qr = reinterpret_cast<uint2 *>(q + row * K);
+    for (int v = lane; v < nvec; v += 32)
+      qr[v] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(xs[v], sc, rc, fast);
+    __syncwarp();  // every lane is done with the slot before it is refilled
+    if (lane == 0 && issued < n_rows) {
+      const int64_t nrow = first + static_cast<int64_t>(issued) * stride;
+      mbar_arrive_expect_tx(&bar[slot], row_bytes);
+      bulk_load_g2s(mine + slot * row_bytes, x + nrow * ldx, row_bytes, &bar[slot]);
+      ++issued;
+    }
+  }
+  if (i < n_rows && lane == 0) {
+    // gave up: let the copies still in flight land before the CTA leaves
+    volatile int never = 0;
+    for (int j = i; j < issued; ++j)
+      mbar_wait(&bar[j % slots], static_cast<uint32_t>(j / slots) & 1u, &never);
+  }
+}
+
+// Rows longer than kQuantBulkMaxK: a group of G threads owns one row (G = 32,
+// one warp, whenever the row fits in 12 vectors per lane).  Each
 // thread issues all of its V 16-byte loads at once (evict-first: the
 // activations are read exactly once), reduces max |x| in registers and across
 // the group (shuffles; shared memory when G > 32), then quantizes its
