@@ -320,8 +320,9 @@ W8A8_API int w8a8_linear_fused_noalloc(const void *x_bf16, int64_t M, int64_t K,
 /*
  * Self-test of the division-free quantization step the kernels use: on the
  * GPU, for every positive finite bf16 row maximum a and every bf16 value x
- * with |x| <= a, compares the code the fast step produces against
- * clamp(rint(x / s), -127, 127) computed with an IEEE division, s = a / 127.
+ * with |x| <= a, compares the code the fast step produces -- in its scalar
+ * form and in the packed fp32x2 form -- against clamp(rint(x / s), -127, 127)
+ * computed with an IEEE division, s = a / 127.
  * counts_dev: device array of 2 unsigned 64-bit integers, zeroed by the call;
  * receives [0] the number of (x, a) pairs checked on the fast step and [1] the
  * number of pairs whose code differs (expected 0).  About 10^9 pairs; takes

@@ -497,16 +497,17 @@ int ensure_smem_limit(int bytes) {
   return W8A8_OK;
 }
 
-// Warps per CTA and row slots per warp of quant_rows_bulk_kernel for rows of
-// K elements: as many warps as fit two slots each in the slot storage (16, 8
-// or 4), then as many slots (up to 4) as fit.
-void quant_bulk_shape(int64_t K, int *warps, int *slots) {
+// Warps per row and row slots per group of quant_rows_bulk_kernel for rows of
+// K elements: at most 3072 elements per warp (1, 2 or 4 warps per row), then
+// as many slots (up to 4) as the slot storage holds for the 16 / G groups.
+void quant_bulk_shape(int64_t K, int *group_warps, int *slots) {
   const int64_t row_bytes = 2 * K;
-  int w = kQuantBulkMaxWarps;
-  while (w > 4 && w * 2 * row_bytes > kQuantBulkSmem) w /= 2;
-  int64_t sl = kQuantBulkSmem / (w * row_bytes);
+  int g = 1;
+  while (g < 4 && g * kQuantBulkWarpElems < K) g *= 2;
+  const int64_t groups = kQuantBulkWarps / g;
+  int64_t sl = kQuantBulkSmem / (groups * row_bytes);
   if (sl > kQuantBulkMaxSlots) sl = kQuantBulkMaxSlots;
-  *warps = w;
+  *group_warps = g;
   *slots = static_cast<int>(sl);
 }
 
@@ -518,16 +519,17 @@ int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q,
     const DeviceInfo *d = nullptr;
     int st = query_device(&d);
     if (st != W8A8_OK) return st;
-    int warps = 0, slots = 0;
-    quant_bulk_shape(K, &warps, &slots);
-    const int smem = warps * slots * static_cast<int>(2 * K);
+    int gw = 0, slots = 0;
+    quant_bulk_shape(K, &gw, &slots);
+    const int groups = kQuantBulkWarps / gw;
+    const int smem = groups * slots * static_cast<int>(2 * K);
     st = ensure_smem_limit<quant_rows_bulk_kernel>(kQuantBulkSmem);
     if (st != W8A8_OK) return st;
-    int64_t grid = cdiv(rows, warps);
+    int64_t grid = cdiv(rows, groups);
     if (grid > d->sms) grid = d->sms;
     return launch_ex(true, quant_rows_bulk_kernel, dim3(static_cast<unsigned>(grid)),
-                     dim3(warps * 32), static_cast<size_t>(smem), stream, xp,
-                     static_cast<int>(rows), static_cast<int>(K), ldx, q, s, slots);
+                     dim3(kQuantBulkWarps * 32), static_cast<size_t>(smem), stream, xp,
+                     static_cast<int>(rows), static_cast<int>(K), ldx, q, s, gw, slots);
   }
   // G threads per row (32 .. 256), each holding V <= kQuantMaxV vectors of
   // 8 bf16 in registers; longer rows take the two-pass kernel.
@@ -761,20 +763,28 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
 }
 
 // Every positive finite bf16 maximum a (blockIdx.x + 1) against every bf16
-// value x with |x| <= a: the fast step's result must equal the IEEE-division
-// path's, bit for bit.
+// value x with |x| <= a: the fast step's result -- scalar, and in the packed
+// fp32x2 form the bulk quantization kernel uses -- must equal the
+// IEEE-division path's, bit for bit.
 __global__ void __launch_bounds__(256) quant_exhaustive_kernel(unsigned long long *counts) {
   const uint32_t abits = blockIdx.x + 1u;  // 0x0001 .. 0x7F7F
   const float a = __uint_as_float(abits << 16);
   const float s = __fdiv_rn(a, 127.0f);
   if (!quant_fast_ok(s)) return;
   const float y = __frcp_rn(s);
+  const float2 neg_s = make_float2(-s, -s), y2 = make_float2(y, y);
   unsigned long long checked = 0, bad = 0;
   for (uint32_t xb = threadIdx.x; xb < 65536u; xb += blockDim.x) {
     if ((xb & 0x7FFFu) > abits) continue;  // |x| > a (also skips Inf and NaN)
     const float x = __uint_as_float(xb << 16);
     ++checked;
-    if (quant_fast(x, s, y) != quant_exact(x, s)) ++bad;
+    const uint32_t want = quant_exact(x, s);
+    if (quant_fast(x, s, y) != want) ++bad;
+    // the packed form: x in every one of the 8 positions of a vector
+    const uint32_t w = xb | (xb << 16);
+    const uint2 codes = quant_vec8_x2(make_uint4(w, w, w, w), neg_s, y2);
+    const uint32_t b = want & 0xFFu;
+    if (codes.x != b * 0x01010101u || codes.y != b * 0x01010101u) ++bad;
   }
   atomicAdd(&counts[0], checked);
   if (bad) atomicAdd(&counts[1], bad);

@@ -83,11 +83,11 @@ __device__ __forceinline__ void gemv_load(const int8_t *__restrict__ wq, int N, 
 }
 
 template <int MT, bool FUSED, bool RAW_OUT>
-__global__ void __launch_bounds__(kGemvThreads) gemv_i8_kernel(const GemvParams p) {
+__global__ void __launch_bounds__(kGemvThreads, 2) gemv_i8_kernel(const GemvParams p) {
   extern __shared__ __align__(16) uint8_t gemv_smem[];
   int8_t *qs = reinterpret_cast<int8_t *>(gemv_smem);  // [M][K]
   __shared__ float sas[kGemvMaxM];
-  __shared__ uint32_t red[kGemvWarps];
+  __shared__ uint32_t red[4][kGemvWarps];
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -106,22 +106,65 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_i8_kernel(const GemvParams 
   grid_dependency_wait();
 
   // ---- 1. activation rows -> shared memory (int8) + scales.  Fused, up to
-  // 4 rows: the whole block works on one row at a time (shortest latency
-  // per row); more rows: one warp per row, 8 rows at once.
+  // 4 rows of up to 4096 elements: the whole block loads every row at once
+  // into registers and reduces all their maxima in one block reduction (the
+  // latency of one row, whatever M); longer rows: one row at a time; more
+  // rows: one warp per row, 8 rows at once.
   if constexpr (FUSED && MT <= 4) {
     const int nvec8 = K >> 3;
-    for (int m = 0; m < p.M; ++m) {
-      const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(m) * p.ldx);
-      float mm = 0.0f;
-      for (int v = tid; v < nvec8; v += kGemvThreads) mm = absmax_vec8(__ldg(xr + v), mm);
-      const float amax = __uint_as_float(block_max_u32(__float_as_uint(mm), red));
-      const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
-      const bool fast = quant_fast_ok(sc);
-      const float rc = fast ? __frcp_rn(sc) : 0.0f;
-      if (tid == 0) sas[m] = sc;
-      uint2 *qrow = reinterpret_cast<uint2 *>(qs + m * K);
-      for (int v = tid; v < nvec8; v += kGemvThreads)
-        qrow[v] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(__ldg(xr + v), sc, rc, fast);
+    if (nvec8 <= 2 * kGemvThreads) {
+      uint4 xv[MT][2];
+      uint32_t mb[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(m) * p.ldx);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int v = tid + j * kGemvThreads;
+          xv[m][j] = (m < p.M && v < nvec8) ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        mb[m] = __float_as_uint(absmax_vec8(xv[m][1], absmax_vec8(xv[m][0], 0.0f)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mb[m] = max(mb[m], __shfl_xor_sync(0xFFFFFFFFu, mb[m], o));
+        if (lane == 0) red[m][warp] = mb[m];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        if (m >= p.M) break;
+        uint32_t a = 0u;
+#pragma unroll
+        for (int w = 0; w < kGemvWarps; ++w) a = max(a, red[m][w]);
+        const float amax = __uint_as_float(a);
+        const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+        const bool fast = quant_fast_ok(sc);
+        const float rc = fast ? __frcp_rn(sc) : 0.0f;
+        if (tid == 0) sas[m] = sc;
+        uint2 *qrow = reinterpret_cast<uint2 *>(qs + m * K);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int v = tid + j * kGemvThreads;
+          if (v < nvec8)
+            qrow[v] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(xv[m][j], sc, rc, fast);
+        }
+      }
+    } else {
+      for (int m = 0; m < p.M; ++m) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(p.x + static_cast<int64_t>(m) * p.ldx);
+        float mm = 0.0f;
+        for (int v = tid; v < nvec8; v += kGemvThreads) mm = absmax_vec8(__ldg(xr + v), mm);
+        const float amax = __uint_as_float(block_max_u32(__float_as_uint(mm), red[0]));
+        const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+        const bool fast = quant_fast_ok(sc);
+        const float rc = fast ? __frcp_rn(sc) : 0.0f;
+        if (tid == 0) sas[m] = sc;
+        uint2 *qrow = reinterpret_cast<uint2 *>(qs + m * K);
+        for (int v = tid; v < nvec8; v += kGemvThreads)
+          qrow[v] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(__ldg(xr + v), sc, rc, fast);
+      }
     }
   } else if constexpr (FUSED) {
     for (int m = warp; m < p.M; m += kGemvWarps)

@@ -203,38 +203,106 @@ __global__ void __launch_bounds__(256) quant_rows_long_kernel(const uint16_t *__
 }
 
 // ---------------------------------------------------------------------------
-// The hot-path kernel for rows of up to kQuantBulkMaxK elements: one CTA per
-// SM, persistent, W warps, each warp owning one row at a time.  Rows reach
-// shared memory by bulk copies (one cp.async.bulk per row), S slots per warp,
-// so each warp has S rows in flight and a CTA W * S * 2K bytes -- the whole
-// CTA's share of a 4352 x 3072 layer is requested at once.  Warp w of CTA c
-// takes rows c * W + w + i * gridDim.x * W, i = 0, 1, ..., so rows complete
-// roughly in order across the GPU.  Per row: max |x| over the slot (bit
-// patterns, warp shuffles), the scale and its reciprocal, then the codes from
-// the slot with the division-free step, 8 bytes per lane per store.  Every
-// slot wait is bounded; on expiry the warp waits for its copies in flight and
-// the kernel returns with the device error word set.
+// The hot-path kernel for rows of up to kQuantBulkMaxK elements: one CTA of 16
+// warps per SM, persistent.  A group of G warps (G = 1, 2 or 4: at most 3072
+// elements per warp) owns one row at a time; rows reach shared memory by bulk
+// copies (one cp.async.bulk per row), S slots per group, so each group has S
+// rows in flight and the CTA 16 / G * S * 2K bytes -- the whole CTA's share of
+// a 4352 x 3072 layer is requested at once.  Group g of CTA c takes rows
+// c * groups + g + i * gridDim.x * groups, i = 0, 1, ..., so rows complete
+// roughly in order across the GPU.  Per row: max |x| on bf16 bit patterns
+// (sign cleared, 16x2 integer maxima), across the group's lanes and warps;
+// the scale and its reciprocal; then the codes with the division-free step in
+// packed fp32x2 arithmetic, 8 bytes per lane per store.  Every slot wait is
+// bounded; on expiry the group waits for its copies in flight and the kernel
+// returns with the device error word set.
 constexpr int kQuantBulkMaxK = 12288;
 constexpr int kQuantBulkSmem = 196608;   // slot storage per CTA
-constexpr int kQuantBulkMaxWarps = 16;
+constexpr int kQuantBulkWarps = 16;
 constexpr int kQuantBulkMaxSlots = 4;
+constexpr int kQuantBulkWarpElems = 3072;  // elements of a row per warp, at most
 
-__global__ void __launch_bounds__(kQuantBulkMaxWarps * 32, 1)
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<uint64_t &>(d))
+      : "l"(reinterpret_cast<const uint64_t &>(a)), "l"(reinterpret_cast<const uint64_t &>(b)),
+        "l"(reinterpret_cast<const uint64_t &>(c)));
+  return d;
+}
+
+__device__ __forceinline__ float2 mul2_rn_q(float2 a, float2 b) {
+  float2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t &>(d))
+      : "l"(reinterpret_cast<const uint64_t &>(a)), "l"(reinterpret_cast<const uint64_t &>(b)));
+  return d;
+}
+
+__device__ __forceinline__ float2 add2_rn_q(float2 a, float2 b) {
+  float2 d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t &>(d))
+      : "l"(reinterpret_cast<const uint64_t &>(a)), "l"(reinterpret_cast<const uint64_t &>(b)));
+  return d;
+}
+
+// max |x| of 8 bf16 as packed 16x2 bit patterns, accumulated into m.
+__device__ __forceinline__ uint32_t absmax_bits8(uint4 v, uint32_t m) {
+  m = max_u16x2(m, v.x & 0x7FFF7FFFu);
+  m = max_u16x2(m, v.y & 0x7FFF7FFFu);
+  m = max_u16x2(m, v.z & 0x7FFF7FFFu);
+  return max_u16x2(m, v.w & 0x7FFF7FFFu);
+}
+
+// The division-free step (quant_fast) on two values at once: each lane of
+// every packed operation is the same separately rounded operation.  neg_s =
+// (-s, -s): x - q0 * s == fma(q0, -s, x), exactly.
+__device__ __forceinline__ uint2 quant_vec8_x2(uint4 v, float2 neg_s, float2 y) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const float2 magic = make_float2(kRintMagic, kRintMagic);
+  uint32_t c[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+    const float2 q0 = mul2_rn_q(x, y);
+    const float2 e = fma2_rn(q0, neg_s, x);
+    const float2 q1 = fma2_rn(e, y, q0);
+    const float2 r = add2_rn_q(q1, magic);
+    c[2 * i] = __float_as_uint(r.x);
+    c[2 * i + 1] = __float_as_uint(r.y);
+  }
+  return pack_codes(c);
+}
+
+__global__ void __launch_bounds__(kQuantBulkWarps * 32, 1)
     quant_rows_bulk_kernel(const uint16_t *__restrict__ x, int rows, int K, int64_t ldx,
-                           int8_t *__restrict__ q, float *__restrict__ s, int slots) {
+                           int8_t *__restrict__ q, float *__restrict__ s, int group_warps,
+                           int slots) {
   extern __shared__ __align__(128) uint8_t quant_slots[];
-  __shared__ uint64_t bars[kQuantBulkMaxWarps * kQuantBulkMaxSlots];
+  __shared__ uint64_t bars[kQuantBulkWarps * kQuantBulkMaxSlots];
+  __shared__ uint32_t red[kQuantBulkWarps];
+  __shared__ int okf[kQuantBulkWarps];
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int warps = blockDim.x >> 5;
+  const int G = group_warps;
+  const int groups = kQuantBulkWarps / G;
+  const int group = warp / G, gw = warp % G;    // gw: this warp's index in its group
+  const bool leader = gw == 0 && lane == 0;
   const uint32_t row_bytes = static_cast<uint32_t>(K) * 2u;
-  uint8_t *mine = quant_slots + static_cast<size_t>(warp) * slots * row_bytes;
-  uint64_t *bar = bars + warp * kQuantBulkMaxSlots;
-  const int stride = static_cast<int>(gridDim.x) * warps;
-  const int first = static_cast<int>(blockIdx.x) * warps + warp;
+  uint8_t *mine = quant_slots + static_cast<size_t>(group) * slots * row_bytes;
+  uint64_t *bar = bars + group * kQuantBulkMaxSlots;
+  const int stride = static_cast<int>(gridDim.x) * groups;
+  const int first = static_cast<int>(blockIdx.x) * groups + group;
   const int n_rows = first < rows ? (rows - first + stride - 1) / stride : 0;
   if (threadIdx.x == 0) abort_flag = 0;
-  if (lane == 0)
+  if (leader)
     for (int j = 0; j < slots; ++j) mbar_init(&bar[j], 1);
   fence_mbarrier_init();
   __syncthreads();
@@ -242,7 +310,7 @@ __global__ void __launch_bounds__(kQuantBulkMaxWarps * 32, 1)
   // kernel, and q / s may still be read by it
   grid_dependency_wait();
   int issued = 0;
-  if (lane == 0) {
+  if (leader) {
     for (; issued < slots && issued < n_rows; ++issued) {
       const int64_t row = first + static_cast<int64_t>(issued) * stride;
       mbar_arrive_expect_tx(&bar[issued], row_bytes);
@@ -251,37 +319,62 @@ __global__ void __launch_bounds__(kQuantBulkMaxWarps * 32, 1)
   }
   grid_dependents_launch();  // the GEMM that follows may start its prologue
   const int nvec = K >> 3;
+  const int gthreads = G * 32;
+  const int t = gw * 32 + lane;   // thread index within the group
   int i = 0;
   for (; i < n_rows; ++i) {
     const int slot = i % slots;
     int ok = mbar_wait(&bar[slot], static_cast<uint32_t>(i / slots) & 1u, &abort_flag) ? 1 : 0;
-    if (!__all_sync(0xFFFFFFFFu, ok)) break;
+    ok = __all_sync(0xFFFFFFFFu, ok);
+    if (G > 1) {  // the group's warps leave together or not at all
+      if (lane == 0) okf[warp] = ok;
+      named_barrier_sync(1 + group, gthreads);
+      for (int w = 0; w < G; ++w) ok &= okf[group * G + w];
+    }
+    if (!ok) break;
     const int64_t row = first + static_cast<int64_t>(i) * stride;
     const uint4 *xs = reinterpret_cast<const uint4 *>(mine + slot * row_bytes);
-    float m0 = 0.0f, m1 = 0.0f;
-    int vi = lane;
-    for (; vi + 32 < nvec; vi += 64) {
-      m0 = absmax_vec8(xs[vi], m0);
-      m1 = absmax_vec8(xs[vi + 32], m1);
+    uint32_t m0 = 0u, m1 = 0u;
+    int vi = t;
+    for (; vi + gthreads < nvec; vi += 2 * gthreads) {
+      m0 = absmax_bits8(xs[vi], m0);
+      m1 = absmax_bits8(xs[vi + gthreads], m1);
     }
-    if (vi < nvec) m0 = absmax_vec8(xs[vi], m0);
-    const float amax = __uint_as_float(warp_max_u32(__float_as_uint(fmaxf(m0, m1)), 32));
+    if (vi < nvec) m0 = absmax_bits8(xs[vi], m0);
+    uint32_t mb = max_u16x2(m0, m1);
+    mb = warp_max_u32(max(mb & 0xFFFFu, mb >> 16), 32);
+    if (G > 1) {  // across the group's warps
+      if (lane == 0) red[warp] = mb;
+      named_barrier_sync(1 + group, gthreads);
+      mb = 0u;
+      for (int w = 0; w < G; ++w) mb = max(mb, red[group * G + w]);
+    }
+    const float amax = __uint_as_float(mb << 16);
     const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
     const bool fast = quant_fast_ok(sc);
     const float rc = fast ? __frcp_rn(sc) : 0.0f;
-    if (lane == 0) s[row] = sc;
+    if (t == 0) s[row] = sc;
     uint2 *qr = reinterpret_cast<uint2 *>(q + row * K);
-    for (int v = lane; v < nvec; v += 32)
-      qr[v] = (sc == 0.0f) ? make_uint2(0u, 0u) : quant_vec8(xs[v], sc, rc, fast);
-    __syncwarp();  // every lane is done with the slot before it is refilled
-    if (lane == 0 && issued < n_rows) {
+    if (sc == 0.0f) {
+      for (int v = t; v < nvec; v += gthreads) qr[v] = make_uint2(0u, 0u);
+    } else if (fast) {
+      const float2 neg_s = make_float2(-sc, -sc), y2 = make_float2(rc, rc);
+#pragma unroll 2
+      for (int v = t; v < nvec; v += gthreads) qr[v] = quant_vec8_x2(xs[v], neg_s, y2);
+    } else {
+      for (int v = t; v < nvec; v += gthreads) qr[v] = quant_vec8(xs[v], sc, rc, false);
+    }
+    // every thread of the group is done with the slot (and with red[])
+    // before the slot is refilled
+    if (G > 1) named_barrier_sync(1 + group, gthreads); else __syncwarp();
+    if (leader && issued < n_rows) {
       const int64_t nrow = first + static_cast<int64_t>(issued) * stride;
       mbar_arrive_expect_tx(&bar[slot], row_bytes);
       bulk_load_g2s(mine + slot * row_bytes, x + nrow * ldx, row_bytes, &bar[slot]);
       ++issued;
     }
   }
-  if (i < n_rows && lane == 0) {
+  if (i < n_rows && leader) {
     // gave up: let the copies still in flight land before the CTA leaves
     volatile int never = 0;
     for (int j = i; j < issued; ++j)
