@@ -235,9 +235,10 @@ class Layer:
         self.i = 0
         plan = w8a8.select(M, N, K)
         self.variant = plan["variant_name"]
-        # GEMV: quantization in its prologue (one launch); GEMMs: the
-        # quantization kernel, then the GEMM
-        self.launches_per_step = 1 if self.variant == "gemv" else 2
+        # GEMVs: quantization in their prologue (one launch); GEMMs and the
+        # tensor-core GEMV: the quantization kernel, then the GEMM
+        self.one_launch = self.variant == "gemv"
+        self.launches_per_step = 1 if self.one_launch else 2
 
     def step(self):
         s = self.sets[self.i]
@@ -512,7 +513,7 @@ def run_ours(args):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
     layer = Layer(case, dev)
-    gemv = layer.variant == "gemv"
+    gemv = layer.one_launch
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     t = timed(layer.step, args.steps, warmup, dist, sampler, graph=gemv)
     status = w8a8.last_device_error()
@@ -535,10 +536,11 @@ def run_ours(args):
     if gemv:
         algo_bytes = 2 * M * K + N * K + 6 * N + 2 * M * N
         achieved = algo_bytes / sec_per_step / 1e9
-        traffic, _ = profile_traffic(f"gemv_i8_{case.name}")
+        kname = "gemv_i8"
+        traffic, _ = profile_traffic(f"{kname}_{case.name}")
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                    "traffic": traffic, "kernel": "gemv_i8 (fused quant prologue)",
+                    "traffic": traffic, "kernel": f"{kname} (fused quantization prologue)",
                     "peak_basis": f"{peaks['source']} HBM copy bandwidth (MEASURED_PEAKS.json)",
                     "algorithmic_bytes_per_launch": algo_bytes,
                     "us_per_launch": round(sec_per_step * 1e6, 2),

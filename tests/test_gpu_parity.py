@@ -201,8 +201,9 @@ def test_linear_strided_output():
 
 # ----------------------------------------------------------------- GEMV (M <= 16)
 
-@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 16])
-@pytest.mark.parametrize("N,K", [(128, 256), (1032, 3072), (64, 12288)])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 16])
+@pytest.mark.parametrize("N,K", [(128, 256), (1032, 3072), (64, 12288), (18432, 3072), (136, 16),
+                                 (520, 2064)])
 def test_gemv_fused_and_unfused(M, N, K):
     x, w, b = synth.make_x(M, K, "normal", M), synth.make_w(N, K, M), synth.make_bias(N, M)
     wq_ref, sw_ref = oracle.quantize_weights(w)
