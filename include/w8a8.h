@@ -110,8 +110,8 @@ typedef struct {
                               128-column tiles (one per pair); else 0 */
     int32_t quant_in_gemm_launch; /* GEMM_PAIR: 1 when w8a8_linear_fused_ex
                               with W8A8_FUSED_ONE_LAUNCH can run the per-token
-                              quantization inside the GEMM launch (given the
-                              full workspace, outside stream capture); else 0 */
+                              quantization inside the GEMM launch (K <= 12288,
+                              given the full workspace); else 0 */
     int32_t k_split;       /* GEMV_TC: CTAs (one cluster) sharing each 128-row
                               weight tile along K, 1..8; else 0 */
 } w8a8_plan;
@@ -217,13 +217,18 @@ W8A8_API int w8a8_linear_fused(const void *x_bf16, int64_t M, int64_t K, int64_t
 
 /*
  * w8a8_linear_fused with options.  W8A8_FUSED_ONE_LAUNCH: on a CTA-pair plan
- * with quant_in_gemm_launch set, a workspace holding the row-block counters
- * (w8a8_workspace_size bytes) and a stream that is not capturing, the pair
- * kernel quantizes x itself: the epilogue warps of all CTAs quantize the rows
- * in row-block order before turning to the epilogues, and each producer waits
- * only for the 128-row block it loads.  One launch instead of two,
- * bit-identical results; on a B200 it measured 6-17% slower than the two
- * launches, so it is not the default.  Otherwise the call is exactly
+ * with quant_in_gemm_launch set (K <= 12288) and a workspace holding the
+ * row-block counters (w8a8_workspace_size bytes), the pair kernel quantizes x
+ * itself: the epilogue warps of all CTAs quantize the rows in row-block
+ * order -- the rows the first round of tiles reads through the not yet used
+ * operand ring (bulk copies), later rows through registers while the first
+ * tiles' MMAs run, taking the epilogue of any finished tile between passes --
+ * and each producer waits only for the 128-row block it loads.  The counters
+ * are cleared on the stream before the launch, so the call may be captured in
+ * a CUDA graph.  One launch instead of two, bit-identical results; on a B200
+ * it measured slower than the two launches (QKV 96 vs 89 us: the quantization
+ * traffic during the first rounds slows the GEMM more than the overlap
+ * saves), so it is not the default.  Otherwise the call is exactly
  * w8a8_linear_fused.  Unknown option bits: W8A8_ERR_INVALID_ARG.
  */
 W8A8_API int w8a8_linear_fused_ex(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,

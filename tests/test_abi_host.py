@@ -259,11 +259,12 @@ def test_selector_is_total_and_consistent(M, KN):
 
 
 def test_quantization_inside_the_gemm_launch_plan():
-    # rows that fit one warp's registers and at most 4 passes of 8 rows per CTA
+    # rows whose bf16 fit one epilogue warp's 24 KB share of the operand ring
     assert w8a8.select(4352, 9216, 3072)["quant_in_gemm_launch"] == 1
     assert w8a8.select(4352, 12288, 3072)["quant_in_gemm_launch"] == 1
-    assert w8a8.select(4352, 3072, 12288)["quant_in_gemm_launch"] == 0   # K > 3072
-    assert w8a8.select(8704, 3072, 3072)["quant_in_gemm_launch"] == 0    # 8 passes
+    assert w8a8.select(4352, 3072, 12288)["quant_in_gemm_launch"] == 1
+    assert w8a8.select(8704, 3072, 3072)["quant_in_gemm_launch"] == 1    # any number of passes
+    assert w8a8.select(4352, 3072, 12304)["quant_in_gemm_launch"] == 0   # K > 12288
     assert w8a8.select(100, 3072, 3072)["quant_in_gemm_launch"] == 0     # not the pair kernel
 
 
@@ -304,7 +305,7 @@ def test_selector_plans_are_valid_for_random_shapes(M, n8, k16):
         assert per >= 24 and per * pairs >= st * kb and st < 2 * pairs
         assert (tiles - st) % pairs == 0
     if p["quant_in_gemm_launch"]:
-        assert K <= 3072 and _cdiv(M, p["grid"] * 8) <= 4
+        assert K <= 12288
 
 
 # --------------------------------------------------------------------------

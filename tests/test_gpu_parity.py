@@ -656,10 +656,15 @@ def _fused_call(x, Wq, s_w, b, y, ws, ws_bytes, q_out=None, s_a_out=None, option
 
 
 # (M, N, K, ldx): the QKV shape, a ragged M (last row block of 67 rows, last
-# pass of 3 rows per CTA group) with K = 3072, a short K (single-vector lanes)
-# and a strided x (ldx > K).
+# pass of 3 rows per CTA group) with K = 3072, a short K (single-vector lanes),
+# a strided x (ldx > K), the FFN down-projection (K = 12288: one bulk-path
+# row per warp, longer register-path rows read twice), eight passes of rows
+# (8704 x 3072 x 3072, the first round's rows through the ring, the rest
+# interleaved with epilogues), a ragged 12288-wide K with two bulk rows per
+# warp, and K = 6144 (two rows in flight per warp's share of the ring).
 FUSED_CASES = [(4352, 9216, 3072, 3072), (1091, 3072, 3072, 3072), (1537, 2048, 3072, 3200),
-               (2048, 2048, 512, 512)]
+               (2048, 2048, 512, 512), (4352, 3072, 12288, 12288), (8704, 3072, 3072, 3072),
+               (2600, 1024, 12288, 12296), (3000, 4096, 6144, 6144)]
 
 
 @pytest.mark.parametrize("M,N,K,ldx", FUSED_CASES)
@@ -670,7 +675,7 @@ def test_quantization_fused_into_pair_launch(M, N, K, ldx):
     oracle on sampled rows."""
     plan = w8a8.select(M, N, K)
     assert plan["variant_name"] == "gemm_pair" and plan["quant_in_gemm_launch"] == 1
-    xb = synth.make_x(M, K, "studentt", 17)
+    xb = synth.make_x(M, K, "gelu" if K > 3072 else "studentt", 17)
     x_full = np.zeros((M, ldx), np.uint16)
     x_full[:, :K] = xb
     x = to_dev(x_full)[:, :K]
@@ -697,6 +702,40 @@ def test_quantization_fused_into_pair_launch(M, N, K, ldx):
     rows = sample_rows(M, seed=17, n_random=32)
     y32, y_ref = oracle.epilogue(oracle.gemm_i32(q_ref[rows], wq), s_ref[rows], sw, b)
     assert check_y(bits_of(y1)[rows], y_ref, y32, "fused launch") == 0
+
+
+def test_quantization_fused_into_pair_launch_replayed_in_a_cuda_graph():
+    """The one-launch layer captured in a CUDA graph (its row-block counters
+    are cleared by a memset node of the same graph) and replayed on new
+    activations each time: every replay must equal the oracle."""
+    M, N, K = 2304, 2048, 3072
+    w = synth.make_w(N, K, 23)
+    wq, sw = oracle.quantize_weights(w)
+    b = synth.make_bias(N, 23)
+    Wq, s_w, bd = torch.from_numpy(wq).cuda(), torch.from_numpy(sw).cuda(), to_dev(b)
+    need = w8a8.workspace_size(M, N, K)
+    ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+    x = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            st = B.w8a8_linear_fused_ex(B._ptr(x), M, K, K, B._ptr(Wq), B._ptr(s_w), B._ptr(bd), N,
+                                        B._ptr(y), N, None, None, B._ptr(ws), need,
+                                        B.FUSED_ONE_LAUNCH, B._stream(s))
+            assert st == 0, B.status_string(st)
+    torch.cuda.current_stream().wait_stream(s)
+    for seed in (31, 32, 33):
+        xb = synth.make_x(M, K, "studentt", seed)
+        x.copy_(to_dev(xb))
+        g.replay()
+        torch.cuda.synchronize()
+        rows = sample_rows(M, seed=seed, n_random=24)
+        r = oracle.linear(np.ascontiguousarray(xb[rows]), wq, sw, b)
+        assert check_y(bits_of(y)[rows], r["y"], r["y32"], f"graph replay {seed}") == 0
+    del g
 
 
 # ----------------------------------------------------------------- W8A16 (weight-only)

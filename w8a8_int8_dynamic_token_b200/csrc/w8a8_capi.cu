@@ -95,11 +95,10 @@ int check_n(int64_t N, int64_t ldy) {
 // ---------------------------------------------------------------- selector
 
 // The fused pair launch quantizes x with its epilogue warps (8 per CTA), one
-// row per warp per pass, before they turn to the epilogues: used when a row
-// fits one warp's registers and at most kFuseMaxPasses passes are needed (more
-// would hold back the first epilogues long enough to stall the MMAs).
-constexpr int64_t kFuseMaxK = 3072;
-constexpr int64_t kFuseMaxPasses = 4;
+// row per warp per pass; the rows the first round of tiles reads come through
+// the operand ring, one row per warp's share of it at least, hence the bound
+// on K (24 KB per warp: 12288 bf16).
+constexpr int64_t kFuseMaxK = 12288;
 
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -233,8 +232,7 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     plan->tile_n = 256;
     plan->num_tiles = static_cast<int32_t>(tiles);
     plan->grid = static_cast<int32_t>(2 * pairs);
-    plan->quant_in_gemm_launch =
-        (K <= kFuseMaxK && cdiv(M, 2 * pairs * kEpiWarps) <= kFuseMaxPasses) ? 1 : 0;
+    plan->quant_in_gemm_launch = K <= kFuseMaxK ? 1 : 0;
     if (nsplit > 1) {
       plan->tail_tiles_nsplit = static_cast<int32_t>(nsplit);
       plan->waves_x100 = static_cast<int32_t>(100 * full + 100 / nsplit);
@@ -600,6 +598,27 @@ int launch_gemm_t(const w8a8_plan &plan, const int8_t *q, const float *s_a, int6
                    mb, my, p);
 }
 
+// Rows of x that the pair kernel's first round of work items reads: every
+// pair's first item is a tile below min(tiles, pairs) in the banded order
+// (or a K-piece of one), so the row blocks of those tiles, rounded to whole
+// 128-row counter blocks and capped at M.
+int64_t pair_first_round_rows(const w8a8_plan &plan, int64_t M, int64_t N) {
+  const int64_t num_m = cdiv(M, 256), num_n = cdiv(N, kPairBN);
+  const int64_t group_m = kGemmGroupM / 2;
+  const int64_t pairs = plan.grid / 2;
+  const int64_t upto = plan.num_tiles < pairs ? plan.num_tiles : pairs;
+  int64_t max_mb = 0;
+  for (int64_t t = 0; t < upto; ++t) {
+    const int64_t band = group_m * num_n;
+    const int64_t g = t / band, first_m = g * group_m;
+    const int64_t rows_in_band = num_m - first_m < group_m ? num_m - first_m : group_m;
+    const int64_t mb = first_m + (t - g * band) % rows_in_band;
+    if (mb > max_mb) max_mb = mb;
+  }
+  const int64_t rows = (max_mb + 1) * 256;
+  return rows < M ? rows : M;
+}
+
 // The per-token quantization fused into the pair launch: x is quantized into
 // q / s_a (the GEMM's operands) by the kernel itself.
 struct FuseArgs {
@@ -675,6 +694,7 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
   p.s_a_w = nullptr;
   p.row_ready = nullptr;
   p.fuse_tag = 0;
+  p.fuse_bulk_rows = 0;
   if (FUSE) {
     p.x = static_cast<const uint16_t *>(fuse->x);
     p.ldx = fuse->ldx;
@@ -682,6 +702,7 @@ int launch_gemm_pair(const w8a8_plan &plan, const int8_t *q, const float *s_a, i
     p.s_a_w = const_cast<float *>(s_a);
     p.row_ready = fuse->row_ready;
     p.fuse_tag = next_tag(48);
+    p.fuse_bulk_rows = static_cast<int32_t>(pair_first_round_rows(plan, M, N));
   }
   constexpr auto kernel = gemm_i8_tcgen05_pair_kernel<kGemmStagesPair, RAW, FUSE>;
   st = ensure_smem_limit<kernel>(L::kSmemBytes);
@@ -1096,18 +1117,10 @@ int w8a8_linear_fused_ex(const void *x, int64_t M, int64_t K, int64_t ldx, const
     split_ws = static_cast<uint8_t *>(workspace) + head;
     split_bytes = ws_bytes - head;
   }
-  // One launch only on request: it measured 6-17% slower than the two
-  // launches, because the 8 epilogue warps of a CTA, quantizing before the
-  // first tiles, keep too few loads in flight to stream x at HBM speed.  Its
-  // counters carry a tag drawn here, on the host: a captured graph would
-  // replay one tag, so under stream capture the two launches are used instead.
-  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
-  if ((options & W8A8_FUSED_ONE_LAUNCH) && cudaStreamIsCapturing(stream, &capture) != cudaSuccess) {
-    cudaGetLastError();
-    return W8A8_ERR_CUDA;
-  }
+  // One launch on request.  Its row-block counters are cleared on the stream
+  // before the launch (a captured graph clears them on every replay).
   if ((options & W8A8_FUSED_ONE_LAUNCH) && plan.variant == W8A8_VARIANT_GEMM_PAIR &&
-      plan.quant_in_gemm_launch && have_ready && capture == cudaStreamCaptureStatusNone) {
+      plan.quant_in_gemm_launch && have_ready) {
     // one launch: the pair kernel quantizes x itself, its producers waiting
     // only for the 128-row blocks they load
     FuseArgs f;

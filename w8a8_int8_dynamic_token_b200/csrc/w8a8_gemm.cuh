@@ -97,22 +97,28 @@ struct GemmParams {
   // resets it to 0.
   unsigned long long *split_counters;
   unsigned long long split_epoch;  // 1 .. 2^56 - 1
-  // CTA-pair kernel with the per-token quantization fused in (K <= 3072: a
-  // row fits one warp's registers): the epilogue warps of all CTAs first
-  // quantize the rows of x (bf16 [M, K], row stride ldx) into q_w / s_a_w --
-  // the buffers the GEMM then reads through tmap_a and s_a.  In pass j, CTA c
-  // takes rows 8 c .. 8 c + 7 + j * 8 * gridDim.x (one per epilogue warp), so
-  // the 128-row blocks complete in order; after each pass one thread of the
-  // CTA adds its rows to the block's counter, (fuse_tag << 16) | rows (the
-  // host clears the counters before the launch, and a counter holding
-  // another launch's tag counts as 0).  A producer waits for its block's
-  // count before loading q.
+  // CTA-pair kernel with the per-token quantization fused in (K <= 12288):
+  // the epilogue warps of all CTAs quantize the rows of x (bf16 [M, K], row
+  // stride ldx) into q_w / s_a_w -- the buffers the GEMM then reads through
+  // tmap_a and s_a.  In pass j, CTA c takes rows 8 c .. 8 c + 7 + j * 8 *
+  // gridDim.x (one per epilogue warp), so the 128-row blocks complete in
+  // order; after each pass one thread of the CTA adds its rows to the block's
+  // counter, (fuse_tag << 16) | rows (the host clears the counters before the
+  // launch, and a counter holding another launch's tag counts as 0).  A
+  // producer waits for its block's count before loading q.  Rows below
+  // fuse_bulk_rows (those the first round of tiles reads) are brought into
+  // the still unused operand ring by bulk copies, every warp's rows at once;
+  // the producer starts filling the ring once every epilogue warp is done
+  // with it.  Later rows are read into registers while the first tiles' MMAs
+  // run, and between passes the warps take the epilogue of any tile whose
+  // accumulator is ready.
   const uint16_t *x;
   int64_t ldx;
   int8_t *q_w;
   float *s_a_w;
   unsigned long long *row_ready;   // cdiv(M, 128) counters
   unsigned long long fuse_tag;     // 1 .. 2^48 - 1
+  int32_t fuse_bulk_rows;          // rows [0, fuse_bulk_rows) take the bulk path
 };
 
 // One epilogue warp slice of a 256 x 256 pair tile: 32 rows x 128 columns.
@@ -618,9 +624,15 @@ struct PairLayout {
   static constexpr int kEpiOffset = kTileBytes;  // 1024-aligned
   static constexpr int kEpiBytes = kEpiWarps * 2 * kEpiBufBytes;
   static constexpr int kBarOffset = kEpiOffset + kEpiBytes;
-  static constexpr int kBarBytes = (2 * STAGES + 5) * 8 + 8;
+  // full[S], empty[S], tfull[2], tempty[2], drain, then two words; then the
+  // fused quantization's barriers: kQuantSlots per epilogue warp, ring_free,
+  // and two decision words
+  static constexpr int kQuantSlots = 4;
+  static constexpr int kBarBytes = (2 * STAGES + 5) * 8 + 8 + (kEpiWarps * kQuantSlots + 1) * 8 + 8;
   static constexpr int kSmemBytes = kBarOffset + kBarBytes + 1024;
   static constexpr int kTmemCols = 2 * kPairBN;
+  // each epilogue warp's share of the ring for the bulk-path rows
+  static constexpr int kQuantWarpBytes = STAGES * kStageBytes / kEpiWarps;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -646,6 +658,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t *drain = tempty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  uint64_t *qbar = drain + 2;                         // [kEpiWarps][kQuantSlots]
+  uint64_t *ring_free = qbar + kEpiWarps * L::kQuantSlots;
+  volatile int *epi_go = reinterpret_cast<volatile int *>(ring_free + 1);  // [2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -664,6 +679,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
+    if constexpr (FUSE_QUANT) {
+      for (int i = 0; i < kEpiWarps * L::kQuantSlots; ++i) mbar_init(&qbar[i], 1);
+      mbar_init(ring_free, kEpiWarps);
+      epi_go[0] = epi_go[1] = 0;
+    }
     fence_mbarrier_init();
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
@@ -699,7 +719,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       auto stage_tx = [&](const WorkItem &it) {
         return 2u * static_cast<uint32_t>(L::kABytes + (it.ncols / 2) * kBK);
       };
-      if (pair_work_item(p, pair_id, num_pairs, 0, w)) {
+      // fused quantization: the epilogue warps use the ring for their first
+      // rows; nothing is loaded into it before they are all done with it
+      if (FUSE_QUANT && !mbar_wait(ring_free, 0u, abort_flag)) ok = false;
+      if (ok && pair_work_item(p, pair_id, num_pairs, 0, w)) {
         int mb0, nb0;
         pair_tile_coords(w.tile, p, mb0, nb0);
         const int nkb = w.kb_end - w.kb_begin;
@@ -816,27 +839,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t acc_phase = 0;
     const int slice = static_cast<int>(rank) * kEpiWarps + e;
     grid_dependency_wait();  // s_a (or, fused, x) comes from the preceding kernel
-    if constexpr (FUSE_QUANT) {
-      // pass j: this CTA's 8 rows 8 c + j * 8 * gridDim.x + e (one 128-row
-      // block: 8 divides 128), then one arrival for all of them
-      const int stride = static_cast<int>(gridDim.x) * kEpiWarps;
-      for (int base = static_cast<int>(blockIdx.x) * kEpiWarps; base < p.M; base += stride) {
-        const int row = base + e;
-        if (row < p.M)
-          quant_row_by_warp<12>(p.x + static_cast<int64_t>(row) * p.ldx, p.K,
-                                p.q_w + static_cast<int64_t>(row) * p.K, p.s_a_w + row, lane);
-        fence_proxy_async_global();
-        __threadfence();  // release: every lane's q and s_a stores before the count
-        named_barrier_sync(1, kEpiWarps * 32);
-        if (e == 0 && lane == 0) {
-          const int rows = p.M - base < kEpiWarps ? p.M - base : kEpiWarps;
-          tagged_arrive<16>(&p.row_ready[base / kBM], p.fuse_tag,
-                            static_cast<unsigned long long>(rows));
-        }
-      }
-    }
-    WorkItem w;
-    for (int it = 0; pair_work_item(p, pair_id, num_pairs, it, w); ++it) {
+    int it = 0;
+    bool more = true;
+    // The epilogue of this pair's next work item (this warp's slice); false
+    // once the pair has none left or a wait gave up.
+    auto do_item = [&]() -> bool {
+      WorkItem w;
+      if (!pair_work_item(p, pair_id, num_pairs, it, w)) return false;
       int mb, nb;
       pair_tile_coords(w.tile, p, mb, nb);
       if constexpr (FUSE_QUANT) {  // acquire this slice's rows (their s_a)
@@ -847,7 +856,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull[acc], acc_phase, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (!ok) break;
+      if (!ok) return false;
       tc_fence_after();
       // this warp: TMEM lane quarter `quarter`, columns [half * ncols / 2, +ncols / 2)
       const int wcols = w.ncols / 2;
@@ -897,7 +906,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         acc = 0;
         acc_phase ^= 1u;
       }
+      ++it;
+      return true;
+    };
+    if constexpr (FUSE_QUANT) {
+      // pass j: this CTA's 8 rows 8 c + j * 8 * gridDim.x + e (one 128-row
+      // block: 8 divides 128), then one arrival for all of them.  Rows below
+      // fuse_bulk_rows come through this warp's share of the ring (bulk
+      // copies, up to kQuantSlots rows in flight); later rows through
+      // registers.  Between passes, one thread looks whether the next tile's
+      // accumulator is ready, and if so the warps take its epilogue first.
+      const int stride = static_cast<int>(gridDim.x) * kEpiWarps;
+      const int cbase = static_cast<int>(blockIdx.x) * kEpiWarps;
+      const int npass = cbase < p.M ? (p.M - cbase + stride - 1) / stride : 0;
+      const uint32_t row_bytes = static_cast<uint32_t>(p.K) * 2u;
+      int nslots = static_cast<int>(L::kQuantWarpBytes / row_bytes);
+      if (nslots > L::kQuantSlots) nslots = L::kQuantSlots;
+      uint8_t *qslot = smem + e * L::kQuantWarpBytes;
+      uint64_t *wbar = qbar + e * L::kQuantSlots;
+      const int bulk_end = p.fuse_bulk_rows < p.M ? p.fuse_bulk_rows : p.M;
+      const int nbulk =
+          cbase + e < bulk_end ? (bulk_end - cbase - e + stride - 1) / stride : 0;
+      int issued = 0;
+      auto issue = [&]() {
+        const int64_t row = cbase + e + static_cast<int64_t>(issued) * stride;
+        const int sl = issued % nslots;
+        mbar_arrive_expect_tx(&wbar[sl], row_bytes);
+        bulk_load_g2s(qslot + sl * row_bytes, p.x + row * p.ldx, row_bytes, &wbar[sl]);
+        ++issued;
+      };
+      if (lane == 0) {
+        while (issued < nslots && issued < nbulk) issue();
+        if (nbulk == 0) mbar_arrive(ring_free);
+      }
+      for (int j = 0; j < npass; ++j) {
+        const int base = cbase + j * stride;
+        const int row = base + e;
+        if (j < nbulk) {
+          const int sl = j % nslots;
+          int ok = mbar_wait(&wbar[sl], static_cast<uint32_t>(j / nslots) & 1u, abort_flag) ? 1 : 0;
+          ok = __all_sync(0xFFFFFFFFu, ok);
+          if (ok)
+            quant_row_from_smem(reinterpret_cast<const uint4 *>(qslot + sl * row_bytes), p.K,
+                                p.q_w + static_cast<int64_t>(row) * p.K, p.s_a_w + row, lane);
+          __syncwarp();  // every lane is done with the slot
+          if (lane == 0) {
+            if (ok && issued < nbulk) issue();
+            if (j == nbulk - 1) mbar_arrive(ring_free);  // this warp is done with the ring
+          }
+        } else if (row < p.M) {
+          quant_row_by_warp<12>(p.x + static_cast<int64_t>(row) * p.ldx, p.K,
+                                p.q_w + static_cast<int64_t>(row) * p.K, p.s_a_w + row, lane);
+        }
+        fence_proxy_async_global();
+        __threadfence();  // release: every lane's q and s_a stores before the count
+        if (e == 0 && lane == 0) epi_go[j & 1] = (more && mbar_try_wait(&tfull[acc], acc_phase)) ? 1 : 0;
+        named_barrier_sync(1, kEpiWarps * 32);
+        if (e == 0 && lane == 0) {
+          const int rows = p.M - base < kEpiWarps ? p.M - base : kEpiWarps;
+          tagged_arrive<16>(&p.row_ready[base / kBM], p.fuse_tag,
+                            static_cast<unsigned long long>(rows));
+        }
+        if (epi_go[j & 1]) more = do_item();
+      }
+      if (lane == 0) {  // after a wait that gave up: let the copies in flight land
+        for (int j = issued > nslots ? issued - nslots : 0; j < issued; ++j) {
+          volatile int never = 0;
+          mbar_wait(&wbar[j % nslots], static_cast<uint32_t>(j / nslots) & 1u, &never);
+        }
+      }
     }
+    while (more) more = do_item();
     if constexpr (!RAW_OUT) {
       if (lane == 0) bulk_wait_all();
       __syncwarp();

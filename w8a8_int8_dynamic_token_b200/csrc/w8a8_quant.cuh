@@ -281,6 +281,37 @@ __device__ __forceinline__ uint2 quant_vec8_x2(uint4 v, float2 neg_s, float2 y) 
   return pack_codes(c);
 }
 
+// One warp quantizes one row of K elements held in shared memory (16-byte
+// aligned) into qr / *s_out: the bulk kernel's per-row step for one warp.
+__device__ __forceinline__ void quant_row_from_smem(const uint4 *xs, int K, int8_t *qr,
+                                                    float *s_out, int lane) {
+  const int nvec = K >> 3;
+  uint32_t m0 = 0u, m1 = 0u;
+  int vi = lane;
+  for (; vi + 32 < nvec; vi += 64) {
+    m0 = absmax_bits8(xs[vi], m0);
+    m1 = absmax_bits8(xs[vi + 32], m1);
+  }
+  if (vi < nvec) m0 = absmax_bits8(xs[vi], m0);
+  uint32_t mb = max_u16x2(m0, m1);
+  mb = warp_max_u32(max(mb & 0xFFFFu, mb >> 16), 32);
+  const float amax = __uint_as_float(mb << 16);
+  const float sc = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
+  const bool fast = quant_fast_ok(sc);
+  const float rc = fast ? __frcp_rn(sc) : 0.0f;
+  if (lane == 0) *s_out = sc;
+  uint2 *qv = reinterpret_cast<uint2 *>(qr);
+  if (sc == 0.0f) {
+    for (int v = lane; v < nvec; v += 32) qv[v] = make_uint2(0u, 0u);
+  } else if (fast) {
+    const float2 neg_s = make_float2(-sc, -sc), y2 = make_float2(rc, rc);
+#pragma unroll 2
+    for (int v = lane; v < nvec; v += 32) qv[v] = quant_vec8_x2(xs[v], neg_s, y2);
+  } else {
+    for (int v = lane; v < nvec; v += 32) qv[v] = quant_vec8(xs[v], sc, rc, false);
+  }
+}
+
 __global__ void __launch_bounds__(kQuantBulkWarps * 32, 1)
     quant_rows_bulk_kernel(const uint16_t *__restrict__ x, int rows, int K, int64_t ldx,
                            int8_t *__restrict__ q, float *__restrict__ s, int group_warps,
