@@ -658,6 +658,8 @@ def extra_components(args, dev, dist, peaks, world, i8_peak=None):
             out[case.name] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
                               "frac_of_nominal_4500": round(ops / t / 1e12 / NOMINAL_INT8_TOPS, 4),
                               "variant": L.variant}
+            out[case.name].update(layer_breakdown(L, steps, dist, peaks))
+            L.i = 0
             layers[case.name] = L
         up, down = layers["ffn_up"], layers["ffn_down"]
 
@@ -678,6 +680,21 @@ def extra_components(args, dev, dist, peaks, world, i8_peak=None):
         out["unpack_int32_weights"] = unpack_component(dev, dist, peaks, steps)
         out["w8a16_qkv"] = w8a16_component(dev, dist, peaks, steps)
     return out
+
+
+def layer_breakdown(L, steps, dist, peaks) -> dict:
+    """The layer's two kernels timed alone (CUDA graphs, same rotation): the
+    GEMM on precomputed q and the per-token quantization."""
+    M, K = L.case.M, L.case.K
+    L.prepare_gemm_only()
+    L.i = 0
+    tg = timed(L.gemm_step, steps, 3, dist, graph=True) / steps
+    L.i = 0
+    tq = timed(L.quant_step, steps, 3, dist, graph=True) / steps
+    qbytes = 3 * M * K + 4 * M
+    return {"gemm_us": round(tg * 1e6, 2), "gemm_TOPS": round(L.case.ops / tg / 1e12, 1),
+            "quant_us": round(tq * 1e6, 2), "quant_GBs": round(qbytes / tq / 1e9, 1),
+            "quant_frac_hbm": round(qbytes / tq / 1e9 / peaks["hbm_gbs"], 4)}
 
 
 def w8a16_component(dev, dist, peaks, steps):
@@ -831,7 +848,9 @@ def dit_block_component(dev, dist, steps):
     per_layer = {}
     for L in layers:
         L.i = 0
-        per_layer[L.case.name] = round(timed(L.step, steps, 3, dist, graph=True) / steps * 1e6, 2)
+        us = round(timed(L.step, steps, 3, dist, graph=True) / steps * 1e6, 2)
+        per_layer[L.case.name] = {"us": us, "frac_of_nominal_4500":
+                                  round(L.case.ops / us / 1e6 / NOMINAL_INT8_TOPS, 4)}
     ops = sum(c.ops for c in synth.DIT_BLOCK)
     res = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 1),
            "us_graph": round(t_graph * 1e6, 2), "TOPS_graph": round(ops / t_graph / 1e12, 1),
