@@ -483,19 +483,46 @@ def measure_i8_peak(dev, dist=None, iters: int = 10000, reps: int = 5) -> dict:
 
 def measure_int_mm(dev, dist=None, n: int = 8192, reps: int = 20) -> dict:
     """Library reference point: torch._int_mm (cuBLASLt int8 GEMM) at n^3,
-    operands resident, the same int8 operation count convention."""
+    operands resident, the same int8 operation count convention; beside it
+    this library's GEMM on the same operands (raw int32 output, as _int_mm
+    returns) and with the bf16 epilogue, timed the same way."""
+    import w8a8_int8_dynamic_token_b200 as w8a8
     a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
-    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev).t()
+    bt = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+    b = bt.t()
     try:
         torch._int_mm(a, b)
     except Exception as e:  # not available in this build: say so
         return {"error": str(e)[:200]}
+    ops = 2.0 * n ** 3
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     t = timed(lambda: torch._int_mm(a, b), reps, 3, dist, sampler) / reps
-    del a, b
+    ones = torch.ones(n, device=dev)
+    acc = torch.empty((n, n), dtype=torch.int32, device=dev)
+    y = torch.empty((n, n), dtype=torch.bfloat16, device=dev)
+    B = w8a8.binding
+    ws = torch.empty((w8a8.workspace_size(n, n, n),), dtype=torch.uint8, device=dev)
+
+    def ours_raw():
+        st = B.w8a8_linear(B._ptr(a), B._ptr(ones), n, n, B._ptr(bt), B._ptr(ones), None, n,
+                           None, n, B._ptr(acc), B._ptr(ws), ws.numel(), B._stream())
+        if st != 0:
+            raise RuntimeError(B.status_string(st))
+
+    def ours_bf16():
+        st = B.w8a8_linear(B._ptr(a), B._ptr(ones), n, n, B._ptr(bt), B._ptr(ones), None, n,
+                           B._ptr(y), n, None, B._ptr(ws), ws.numel(), B._stream())
+        if st != 0:
+            raise RuntimeError(B.status_string(st))
+
+    t_raw = timed(ours_raw, reps, 3, dist) / reps
+    t_bf16 = timed(ours_bf16, reps, 3, dist) / reps
+    del a, b, bt, acc, y, ws
     torch.cuda.empty_cache()
-    return {"tops": round(2.0 * n ** 3 / t / 1e12, 1), "us": round(t * 1e6, 1), "n": n,
-            "sm_mhz": sampler.summary().get("sm_mhz")}
+    return {"tops": round(ops / t / 1e12, 1), "us": round(t * 1e6, 1), "n": n,
+            "sm_mhz": sampler.summary().get("sm_mhz"),
+            "ours_int32_out_tops": round(ops / t_raw / 1e12, 1),
+            "ours_bf16_out_tops": round(ops / t_bf16 / 1e12, 1)}
 
 
 def run_ours(args):
@@ -752,14 +779,15 @@ def sweep_component(dev, dist, peaks, i8_peak, oracle_rows: int = 4):
             t = timed(L.step, steps, 3, dist, graph=True) / steps
             algo = 2 * M * K + N * K + 6 * N + 2 * M * N
             ai = ops / algo
-            attain = min(i8_peak * 1e12 if i8_peak else NOMINAL_INT8_TOPS * 1e12, ai * bw)
+            peak_ops = i8_peak * 1e12 if i8_peak else NOMINAL_INT8_TOPS * 1e12
+            attain = min(peak_ops, ai * bw)
             rows = min(M, oracle_rows)
             t0 = time.perf_counter()
             oracle.linear(x_bits[:rows], wq_h, sw_h, case.b())
             t_or = time.perf_counter() - t0
             points.append({"M": M, "K": K, "N": N, "variant": L.variant, "us": round(t * 1e6, 2),
                            "TOPS": round(ops / t / 1e12, 1), "GBs": round(algo / t / 1e9, 1),
-                           "bound": "tensor" if ai * bw > attain * 0.999 else "hbm",
+                           "bound": "hbm" if ai * bw < peak_ops else "tensor",
                            "frac_of_attainable": round(ops / t / attain, 4),
                            "frac_of_nominal_4500": round(ops / t / 1e12 / NOMINAL_INT8_TOPS, 4),
                            "oracle_TOPS": round(2.0 * rows * N * K / t_or / 1e12, 5),
