@@ -235,9 +235,9 @@ class Layer:
         self.i = 0
         plan = w8a8.select(M, N, K)
         self.variant = plan["variant_name"]
-        # GEMVs: quantization in their prologue (one launch); GEMMs and the
-        # tensor-core GEMV: the quantization kernel, then the GEMM
-        self.one_launch = self.variant == "gemv"
+        # the GEMV at 1-2 rows: quantization in its prologue (one launch);
+        # otherwise the quantization kernel, then the GEMV or GEMM
+        self.one_launch = self.variant == "gemv" and plan["quant_in_gemm_launch"] == 1
         self.launches_per_step = 1 if self.one_launch else 2
 
     def step(self):

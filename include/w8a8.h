@@ -111,7 +111,10 @@ typedef struct {
     int32_t quant_in_gemm_launch; /* GEMM_PAIR: 1 when w8a8_linear_fused_ex
                               with W8A8_FUSED_ONE_LAUNCH can run the per-token
                               quantization inside the GEMM launch (K <= 12288,
-                              given the full workspace); else 0 */
+                              given the full workspace); GEMV: 1 when
+                              w8a8_linear_fused quantizes the rows inside the
+                              GEMV launch (M = 1, or M = 2 with K <= 8192;
+                              no workspace needed); else 0 */
     int32_t k_split;       /* GEMV_TC: CTAs (one cluster) sharing each 128-row
                               weight tile along K, 1..8; else 0 */
 } w8a8_plan;
@@ -162,7 +165,8 @@ W8A8_API int w8a8_quant_act(const void *x_bf16, int64_t M, int64_t K, int64_t ld
  * it: a call that uses counters clears them on its stream first (an
  * asynchronous memset of a few KB; nothing is allocated).  A workspace
  * holding only q and s_a still works: the layer then runs without the K
- * split.
+ * split.  0 when the plan is the GEMV quantizing its own rows (M = 1, or
+ * M = 2 with K <= 8192).
  */
 W8A8_API int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes);
 
@@ -204,7 +208,9 @@ W8A8_API int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_
  * recommended).  Required: the bytes for q and s_a, unless both q_out and
  * s_a_out are given; the rest (row-block counters, K-split region) is
  * optional, see w8a8_workspace_size.  Two launches: the quantization kernel,
- * then the GEMM as a programmatic dependent launch.
+ * then the GEMM (or the small-M variant the selector picks) as a programmatic
+ * dependent launch; one launch when the plan is the GEMV quantizing its own
+ * rows (w8a8_plan.quant_in_gemm_launch on a GEMV plan).
  */
 W8A8_API int w8a8_linear_fused(const void *x_bf16, int64_t M, int64_t K, int64_t ldx,
                       const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,

@@ -100,16 +100,31 @@ def _golden(name):
 def test_selector_small_m_goes_to_gemv():
     # The AdaLN modulation layer runs at M = batch (1, or 2 with CFG), below
     # the 16 rows a torch._int_mm path cannot serve: every such M is served
-    # here, by the GEMV up to 4 rows (measured crossover) and by the tcgen05
-    # GEMM above.
+    # here, by the GEMV (quantizing its rows in the same launch at M = 1, 2),
+    # from 4 rows on this 18432-wide weight by the tensor-core small-M
+    # variant (measured crossovers), and by the tcgen05 GEMM above.
     g = _golden("int_mm_min_rows.txt")
     lim, K, N = g["int_mm_min_rows_exclusive"], g["adaln_in_features"], g["adaln_out_features"]
-    for M in (1, 2, 4):
-        assert w8a8.select(M, N, K)["variant_name"] == "gemv"
-    for M in (5, lim, lim + 1):
-        assert w8a8.select(M, N, K)["variant_name"].startswith("gemm")
+    for M in (1, 2, 3):
+        p = w8a8.select(M, N, K)
+        assert p["variant_name"] == "gemv" and p["quant_in_gemm_launch"] == int(M <= 2)
+    for M in (4, 5, lim):
+        assert w8a8.select(M, N, K)["variant_name"] == "gemv_tc"
+    assert w8a8.select(lim + 1, N, K)["variant_name"].startswith("gemm")
     assert w8a8.select(lim, N, K, variant=B.VARIANT_GEMV)["variant_name"] == "gemv"
     assert w8a8.workspace_size(1, N, K) == 0
+    assert w8a8.workspace_size(3, N, K) >= 3 * K + 3 * 4   # q and s_a for the quantization kernel
+
+
+def test_selector_narrow_weights_keep_the_gemv_to_16_rows():
+    # 3072 x 3072: the GEMV's dot products stay cheaper than the tensor-core
+    # paths up to 16 rows; 3072 x 12288: the tensor-core variant from 9 rows
+    for M in (3, 8, 16):
+        p = w8a8.select(M, 3072, 3072)
+        assert p["variant_name"] == "gemv" and p["quant_in_gemm_launch"] == 0
+    assert w8a8.select(2, 3072, 12288)["quant_in_gemm_launch"] == 0   # K > 8192: two launches
+    assert w8a8.select(8, 3072, 12288)["variant_name"] == "gemv"
+    assert w8a8.select(9, 3072, 12288)["variant_name"] == "gemv_tc"
 
 
 def test_selector_one_row_block_narrow_n_takes_64_column_tiles():
@@ -130,7 +145,8 @@ def test_selector_gemm_plans():
     p = w8a8.select(64, 128, 256)
     assert p["grid"] == p["num_tiles"] <= 2
     # GEMV would need more than 227 KB of shared memory: falls back to GEMM
-    assert w8a8.select(16, 64, 16384)["variant_name"].startswith("gemm")
+    assert w8a8.select(16, 64, 16384)["variant_name"] == "gemv_tc"
+    assert w8a8.select(17, 64, 16384)["variant_name"].startswith("gemm")
     # forced variants
     assert w8a8.select(1, 64, 256, variant=B.VARIANT_GEMM_BN128)["tile_n"] == 128
     with pytest.raises(w8a8.W8A8Error):
@@ -285,9 +301,17 @@ def test_selector_plans_are_valid_for_random_shapes(M, n8, k16):
     v = p["variant_name"]
     assert p["grid"] >= 1
     if v == "gemv":
-        assert M <= 4 and M * K + 1024 <= 232448
+        assert M <= 16 and M * K + 1024 <= 232448
+        assert not ((M >= 5 and N >= 6144) or (M >= 4 and N >= 16384) or (M >= 9 and K >= 8192))
+        assert p["quant_in_gemm_launch"] == int(M == 1 or (M == 2 and K <= 8192))
         return
     tm, tn, tiles = p["tile_m"], p["tile_n"], p["num_tiles"]
+    if v == "gemv_tc":
+        assert 4 <= M <= 16 and (N >= 6144 or K >= 8192)
+        assert tm == 128 and tn == 16 and tiles == _cdiv(N, 128)
+        ks = p["k_split"]
+        assert 1 <= ks <= 8 and ks <= _cdiv(K, 128) and p["grid"] == tiles * ks
+        return
     assert tiles == _cdiv(M, tm) * _cdiv(N, tn)
     assert p["grid"] <= 148
     if v != "gemm_pair":

@@ -209,9 +209,14 @@ def test_gemv_fused_and_unfused(M, N, K):
     wq_ref, sw_ref = oracle.quantize_weights(w)
     ref = oracle.linear(x, wq_ref, sw_ref, b)
     Wq, s_w = torch.from_numpy(wq_ref).cuda(), torch.from_numpy(sw_ref).cuda()
-    # the selector takes the GEMV up to 4 rows; above, linear_fused runs the
-    # GEMM and the GEMV is checked through its explicit (unfused) variant
-    assert (w8a8.select(M, N, K)["variant_name"] == "gemv") == (M <= 4)
+    # the selector takes the CUDA-core GEMV (quantizing its rows in the same
+    # launch at M = 1, 2) unless the tensor-core variant streams a wide or deep
+    # weight faster; the CUDA-core GEMV is also checked through its explicit
+    # (unfused) variant
+    p = w8a8.select(M, N, K)
+    wide = (M >= 5 and N >= 6144) or (M >= 4 and N >= 16384) or (M >= 9 and K >= 8192)
+    assert p["variant_name"] == ("gemv_tc" if wide else "gemv")
+    assert p["quant_in_gemm_launch"] == (0 if wide else int(M == 1 or (M == 2 and K <= 8192)))
     y, q, s_a = w8a8.linear_fused(to_dev(x), Wq, s_w, to_dev(b), return_intermediates=True)
     y2 = w8a8.linear_fused(to_dev(x), Wq, s_w, to_dev(b))
     y3 = w8a8.linear(torch.from_numpy(ref["q"]).cuda(), torch.from_numpy(ref["s_a"]).cuda(), Wq,
@@ -255,6 +260,27 @@ def test_gemv_tc_int32_exact_and_y(M, N, K):
     assert check_y(bits_of(y), ref["y"], ref["y32"], "gemv_tc") == 0
     y32n, yn = oracle.epilogue(ref["acc"], ref["s_a"], sw_ref, None)
     assert check_y(bits_of(y_nobias), yn, y32n, "gemv_tc no bias") == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(6, 136, 40000), (16, 3072, 12288), (11, 9216, 3072)])
+def test_small_m_whole_layer_with_intermediates(M, N, K):
+    """linear_fused at 5 <= M <= 16 against a deep or wide weight: the
+    quantization kernel, then the tensor-core small-M variant reading q (K
+    shared among up to 8 CTAs of a cluster): y, q and s_a against the oracle
+    in full."""
+    x, w, b = synth.make_x(M, K, "studentt", M + 40), synth.make_w(N, K, M + 40), synth.make_bias(N, M + 40)
+    wq_ref, sw_ref = oracle.quantize_weights(w)
+    ref = oracle.linear(x, wq_ref, sw_ref, b)
+    Wq, s_w = torch.from_numpy(wq_ref).cuda(), torch.from_numpy(sw_ref).cuda()
+    assert w8a8.select(M, N, K)["variant_name"] == "gemv_tc"
+    y, q, s_a = w8a8.linear_fused(to_dev(x), Wq, s_w, to_dev(b), return_intermediates=True)
+    y2 = w8a8.linear_fused(to_dev(x), Wq, s_w, None)
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), ref["q"])
+    assert np.array_equal(f32_bits(s_a.cpu().numpy()), f32_bits(ref["s_a"]))
+    assert check_y(bits_of(y), ref["y"], ref["y32"], "small-M layer") == 0
+    y32n, yn = oracle.epilogue(ref["acc"], ref["s_a"], sw_ref, None)
+    assert check_y(bits_of(y2), yn, y32n, "small-M layer, no bias") == 0
 
 
 def test_gemv_tc_extremes_at_max_k():

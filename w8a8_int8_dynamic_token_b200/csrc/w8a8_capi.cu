@@ -18,7 +18,7 @@
 #include "w8a8_gemv.cuh"
 #include "w8a8_pack.cuh"
 #include "w8a8_peak.cuh"
-#include "w8a16_gemm.cuh"
+#include "w8a16_tmem.cuh"
 #include "w8a8_ptx.cuh"
 #include "w8a8_quant.cuh"
 #include "w8a8_swapab.cuh"
@@ -107,15 +107,35 @@ inline bool gemv_fits(int64_t M, int64_t K, int max_smem) {
   return M <= kGemvMaxM && M * K + 1024 <= static_cast<int64_t>(max_smem);
 }
 
-// The selector takes the GEMV up to this many rows.  Measured on a B200 (the
-// whole layer, CUDA graphs): the GEMV streams the weight at 4-5 TB/s at M = 1
-// and its per-row dot products cost about 1.8 us per extra row at N = 9216,
-// K = 3072, while the tcgen05 GEMM path costs 12-16 us flat for M <= 128
-// there (launch, pipeline fill and epilogue bound); they cross at M = 5-6.
-constexpr int64_t kGemvAutoMaxM = 4;
-
 // The tensor-core small-M variant serves up to this many activation rows.
 constexpr int64_t kSwapMaxM = 128;
+
+// Small-M selection, from whole-layer times on a B200 (quantization
+// included, CUDA graphs of back-to-back calls; us):
+//
+//   N x K          M:   1     2     4     5     8    12    16
+//   18432 x 3072  gemv 10.3* 11.9* 15.8  19.2  22.9  30.4  34.6
+//                 tc   14.1  14.1  14.4  15.1  15.7  16.5  17.3   GEMM 18.8-19.5
+//   9216 x 3072   gemv  6.3*  7.5* 10.1  12.0  14.2  18.0  20.6
+//                 tc   10.4  10.7  11.0  11.4  12.0  13.0  13.9   GEMM 14.2-15.1
+//   3072 x 3072   gemv  3.6*  4.1*  5.9   7.2   8.5  11.1  12.8
+//                 tc   13.4  13.6  14.0  14.3  14.9  16.0  17.0   GEMM 11.6-12.8
+//   3072 x 12288  gemv  9.2*  11.3  14.1  16.9  20.8  37.7  43.9
+//                 tc   21.3  22.3  22.9  23.0  23.5  24.2  24.8   GEMM 30.4-32.1
+//
+// (* the GEMV with the quantization in its own launch; elsewhere the
+// quantization kernel runs first.)  The GEMV's dot products cost 1-2 us per
+// row on wide weights; the tensor-core variant is flat in M but pays for its
+// cluster-shared K on narrow ones.
+inline bool gemv_quantizes_itself(int64_t M, int64_t K) { return M == 1 || (M == 2 && K <= 8192); }
+inline bool swap_beats_gemv(int64_t M, int64_t N, int64_t K) {
+  return (M >= 5 && N >= 6144) || (M >= 4 && N >= 16384) || (M >= 9 && K >= 8192);
+}
+// Without the GEMV (K too deep for its shared-memory rows), the tensor-core
+// variant still beats one row block of the GEMM on wide or deep weights.
+constexpr int64_t kSwapAutoMaxM = 16;
+constexpr int64_t kSwapAutoMinN = 6144;
+constexpr int64_t kSwapAutoMinK = 8192;
 
 inline int swap_mpad(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
 
@@ -133,8 +153,14 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
   if (sms < 1) return W8A8_ERR_INVALID_ARG;
   int v = variant;
   if (v == W8A8_VARIANT_AUTO) {
-    if (M <= kGemvAutoMaxM && gemv_fits(M, K, max_smem)) {
+    if (gemv_fits(M, K, max_smem) && !swap_beats_gemv(M, N, K)) {
       v = W8A8_VARIANT_GEMV;
+    } else if (M <= kSwapAutoMaxM && (N >= kSwapAutoMinN || K >= kSwapAutoMinK)) {
+      // a handful of rows against a wide or deep weight: the tensor-core
+      // small-M variant (its K shared among the CTAs of a cluster) streams
+      // the weight faster than the GEMV's dot products or one row block of
+      // the GEMM
+      v = W8A8_VARIANT_GEMV_TC;
     } else if (M <= kBM && cdiv(N, 128) * 3 <= sms) {
       // one row block and few 128-column tiles: 64-column tiles put twice as
       // many CTAs on the weight stream (measured ~4% faster at N = 3072)
@@ -193,6 +219,7 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     const int64_t cap = static_cast<int64_t>(sms) * per_sm;
     plan->num_tiles = static_cast<int32_t>(N);
     plan->grid = static_cast<int32_t>(grid < cap ? grid : cap);
+    plan->quant_in_gemm_launch = gemv_quantizes_itself(M, K) ? 1 : 0;
     return W8A8_OK;
   }
   if (v == W8A8_VARIANT_GEMM_PAIR) {
@@ -382,7 +409,7 @@ int encode_bf16_load_map(CUtensorMap *map, const void *base, int64_t rows, int64
   if (enc == nullptr) return W8A8_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kW16BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kWtBK), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -390,18 +417,19 @@ int encode_bf16_load_map(CUtensorMap *map, const void *base, int64_t rows, int64
   return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
 }
 
-// int8 matrix [rows, K] dense, box 64 (K) x box_rows, no swizzle (the W8A16
-// GEMM's weights, widened to bf16 in shared memory by the kernel).
-int encode_i8_plain_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K,
-                        int box_rows) {
+// int8 matrix [rows, K] dense, box 64 (K) x box_rows, 64-byte swizzle (the
+// tensor-memory W8A16 GEMM's weights: a converter lane reads one row's four
+// 16-byte chunks without bank conflicts).
+int encode_i8_sw64_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K,
+                       int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
   if (enc == nullptr) return W8A8_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kW16BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kWtBK), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
 }
@@ -1029,7 +1057,7 @@ int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes) {
   w8a8_plan plan;
   st = select_plan(M, N, K, 148, W8A8_VARIANT_AUTO, 232448, &plan);
   if (st != W8A8_OK) return st;
-  *bytes = plan.variant == W8A8_VARIANT_GEMV
+  *bytes = plan.variant == W8A8_VARIANT_GEMV && plan.quant_in_gemm_launch
                ? 0
                : fused_workspace_bytes(M, K) + ready_counter_bytes(M) +
                      split_workspace_bytes(plan);
@@ -1082,7 +1110,7 @@ int w8a8_linear_fused_ex(const void *x, int64_t M, int64_t K, int64_t ldx, const
   st = select_plan(M, N, K, d->sms, W8A8_VARIANT_AUTO, d->max_smem_optin, &plan);
   if (st != W8A8_OK) return st;
 
-  if (plan.variant == W8A8_VARIANT_GEMV) {
+  if (plan.variant == W8A8_VARIANT_GEMV && plan.quant_in_gemm_launch) {
     GemvParams p = {};
     p.M = static_cast<int32_t>(M);
     p.N = static_cast<int32_t>(N);
@@ -1212,41 +1240,33 @@ int w8a16_linear(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t 
   const DeviceInfo *d = nullptr;
   st = query_device(&d);
   if (st != W8A8_OK) return st;
-  constexpr int BN = 128, STAGES = 4;
-  using L = W16Layout<BN, STAGES>;
-  CUtensorMap mx, mw, my;
-  st = encode_bf16_load_map(&mx, x, M, K, ldx, kBM);
+  using L = WtLayout;
+  CUtensorMap mx, mw;
+  st = encode_bf16_load_map(&mx, x, M, K, ldx, kWtBN);
   if (st != W8A8_OK) return st;
-  st = encode_i8_plain_map(&mw, Wq, N, K, BN);
+  st = encode_i8_sw64_map(&mw, Wq, N, K, kBM);
   if (st != W8A8_OK) return st;
-  st = encode_bf16_store_map(&my, y, M, N, ldy);
-  if (st != W8A8_OK) return st;
-  GemmParams p;
+  WtParams p;
   std::memset(&p, 0, sizeof(p));
   p.M = static_cast<int32_t>(M);
   p.N = static_cast<int32_t>(N);
   p.K = static_cast<int32_t>(K);
-  p.num_m_blk = static_cast<int32_t>(cdiv(M, kBM));
-  p.num_n_blk = static_cast<int32_t>(cdiv(N, BN));
+  p.num_n_blk = static_cast<int32_t>(cdiv(N, kBM));
+  p.num_m_blk = static_cast<int32_t>(cdiv(M, kWtBN));
   const int64_t tiles = static_cast<int64_t>(p.num_m_blk) * p.num_n_blk;
   if (tiles > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
   p.num_tiles = static_cast<int32_t>(tiles);
-  p.k_blocks = static_cast<int32_t>(cdiv(K, kW16BK));
-  p.group_m = kGemmGroupM;
-  p.s_a = nullptr;
+  p.k_blocks = static_cast<int32_t>(cdiv(K, kWtBK));
   p.s_w = s_w;
   p.bias = static_cast<const uint16_t *>(bias);
   p.y = static_cast<uint16_t *>(y);
   p.ldy = ldy;
-  p.acc_out = nullptr;
-  p.dp_tiles = p.num_tiles;
-  p.tail_nsplit = 1;
-  constexpr auto kernel = gemm_w8a16_tcgen05_kernel<BN, STAGES>;
+  constexpr auto kernel = gemm_w8a16_tmem_kernel;
   st = ensure_smem_limit<kernel>(L::kSmemBytes);
   if (st != W8A8_OK) return st;
   const int64_t grid = tiles < d->sms ? tiles : d->sms;
-  return launch_ex(true, kernel, dim3(static_cast<unsigned>(grid)), dim3(kW16Threads),
-                   L::kSmemBytes, reinterpret_cast<cudaStream_t>(stream), mx, mw, my, p);
+  return launch_ex(true, kernel, dim3(static_cast<unsigned>(grid)), dim3(kWtThreads),
+                   L::kSmemBytes, reinterpret_cast<cudaStream_t>(stream), mx, mw, p);
 }
 
 int w8a8_last_device_error(w8a8_stream_t stream) {

@@ -76,6 +76,89 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t local, uint32_t rank, uin
                : "memory");
 }
 
+// The epilogue of both kernels (warps 2..5, TMEM lane quarter warp & 3, i.e.
+// 32 weight rows n of the tile each), after the MMAs of every CTA of the
+// cluster: the other CTAs store their int32 partial sums into the first
+// CTA's idle ring (distributed shared memory), which adds them exactly and
+// writes y[m, n] = bf16_rne(((float)acc * s_a[m]) * s_w[n] + (float)bias[n]).
+// s_a: the row scales, written by the preceding kernel.  All threads of the
+// CTA call it.
+template <int MPAD, bool RAW_OUT>
+__device__ __forceinline__ void swap_epilogue(const SwapParams &p, uint32_t tmem_base,
+                                              uint64_t *tfull, volatile int *abort_flag,
+                                              uint8_t *ring, int warp, int lane, int tile,
+                                              int rank, int split, const float *s_a) {
+  const bool epi = warp >= 2;
+  const int quarter = warp & 3;
+  const int row_local = quarter * 32 + lane;          // 0..127 within the tile
+  const int n = tile * kBM + row_local;
+  int ok = 1;
+  if (epi) {
+    ok = mbar_wait(tfull, 0u, abort_flag) ? 1 : 0;
+    tc_fence_after();
+  }
+  // every CTA's MMAs have completed: the first CTA's ring may take partials
+  __syncwarp();
+  if (split > 1) cluster_sync();
+  const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+  uint8_t *partials = ring;  // [rank - 1][row_local][MPAD] int32, in the first CTA
+  // columns per TMEM load: 32, or MPAD when it is 16 (32 are allocated)
+  constexpr int CW = MPAD < 32 ? MPAD : 32;
+  if (split > 1 && epi && rank > 0 && ok) {
+#pragma unroll 1
+    for (int c = 0; c < MPAD; c += CW) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(t_row + c, r);
+      tmem_ld_wait();
+      const uint32_t base = smem_addr(partials + (static_cast<size_t>(rank - 1) * kBM + row_local) *
+                                                     MPAD * 4 + c * 4);
+#pragma unroll
+      for (int g = 0; g < CW / 4; ++g)
+        st_cluster_v4(base + 16u * g, 0u,
+                      make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]));
+    }
+  }
+  if (split > 1) cluster_sync();  // partials visible in the first CTA
+  if (epi && rank == 0 && ok) {
+    grid_dependency_wait();  // s_a comes from the preceding kernel
+    const bool n_ok = n < p.N;
+    const float sw = n_ok ? __ldg(p.s_w + n) : 0.0f;
+    const float bv = (n_ok && p.bias != nullptr)
+                         ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16)
+                         : 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < MPAD; c += CW) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(t_row + c, r);
+      tmem_ld_wait();
+      for (int j = 1; j < split; ++j) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            partials + (static_cast<size_t>(j - 1) * kBM + row_local) * MPAD * 4 + c * 4);
+#pragma unroll
+        for (int g = 0; g < CW / 4; ++g) {
+          const uint4 a = src[g];
+          r[4 * g] += a.x; r[4 * g + 1] += a.y; r[4 * g + 2] += a.z; r[4 * g + 3] += a.w;
+        }
+      }
+      if (!n_ok) continue;
+#pragma unroll
+      for (int j = 0; j < CW; ++j) {
+        const int m = c + j;
+        if (m >= p.M) break;
+        if constexpr (RAW_OUT) {
+          p.acc_out[static_cast<int64_t>(m) * p.N + n] = static_cast<int32_t>(r[j]);
+        } else {
+          float v = __int2float_rn(static_cast<int32_t>(r[j]));
+          v = __fmul_rn(__fmul_rn(v, __ldcg(s_a + m)), sw);
+          if (p.bias != nullptr) v = __fadd_rn(v, bv);
+          const __nv_bfloat16 h = __float2bfloat16_rn(v);
+          p.y[static_cast<int64_t>(m) * p.ldy + n] = *reinterpret_cast<const uint16_t *>(&h);
+        }
+      }
+    }
+  }
+}
+
 template <int MPAD, bool RAW_OUT>
 __global__ void __launch_bounds__(kSwThreads, 1)
     gemm_i8_swapab_kernel(const __grid_constant__ CUtensorMap tmap_w,
@@ -197,76 +280,8 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   }
 
   // ---------------------------------------------------------------- epilogue
-  // warps 2..5: TMEM lane quarter (warp & 3), i.e. weight rows n of the tile
-  const bool epi = warp >= 2;
-  const int quarter = warp & 3;
-  const int row_local = quarter * 32 + lane;          // 0..127 within the tile
-  const int n = tile * kBM + row_local;
-  int ok = 1;
-  if (epi) {
-    ok = mbar_wait(tfull, 0u, abort_flag) ? 1 : 0;
-    tc_fence_after();
-  }
-  // every CTA's MMAs have completed: the first CTA's ring may take partials
-  __syncwarp();
-  if (split > 1) cluster_sync();
-  const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-  uint8_t *partials = smem;  // [rank - 1][row_local][MPAD] int32, in the first CTA
-  // columns per TMEM load: 32, or MPAD when it is 16 (32 are allocated)
-  constexpr int CW = MPAD < 32 ? MPAD : 32;
-  if (split > 1 && epi && rank > 0 && ok) {
-#pragma unroll 1
-    for (int c = 0; c < MPAD; c += CW) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(t_row + c, r);
-      tmem_ld_wait();
-      const uint32_t base = smem_addr(partials + (static_cast<size_t>(rank - 1) * kBM + row_local) *
-                                                     MPAD * 4 + c * 4);
-#pragma unroll
-      for (int g = 0; g < CW / 4; ++g)
-        st_cluster_v4(base + 16u * g, 0u,
-                      make_uint4(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3]));
-    }
-  }
-  if (split > 1) cluster_sync();  // partials visible in the first CTA
-  if (epi && rank == 0 && ok) {
-    grid_dependency_wait();  // s_a comes from the preceding kernel
-    const bool n_ok = n < p.N;
-    const float sw = n_ok ? __ldg(p.s_w + n) : 0.0f;
-    const float bv = (n_ok && p.bias != nullptr)
-                         ? __uint_as_float(static_cast<uint32_t>(__ldg(p.bias + n)) << 16)
-                         : 0.0f;
-#pragma unroll 1
-    for (int c = 0; c < MPAD; c += CW) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(t_row + c, r);
-      tmem_ld_wait();
-      for (int j = 1; j < split; ++j) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            partials + (static_cast<size_t>(j - 1) * kBM + row_local) * MPAD * 4 + c * 4);
-#pragma unroll
-        for (int g = 0; g < CW / 4; ++g) {
-          const uint4 a = src[g];
-          r[4 * g] += a.x; r[4 * g + 1] += a.y; r[4 * g + 2] += a.z; r[4 * g + 3] += a.w;
-        }
-      }
-      if (!n_ok) continue;
-#pragma unroll
-      for (int j = 0; j < CW; ++j) {
-        const int m = c + j;
-        if (m >= p.M) break;
-        if constexpr (RAW_OUT) {
-          p.acc_out[static_cast<int64_t>(m) * p.N + n] = static_cast<int32_t>(r[j]);
-        } else {
-          float v = __int2float_rn(static_cast<int32_t>(r[j]));
-          v = __fmul_rn(__fmul_rn(v, __ldcg(p.s_a + m)), sw);
-          if (p.bias != nullptr) v = __fadd_rn(v, bv);
-          const __nv_bfloat16 h = __float2bfloat16_rn(v);
-          p.y[static_cast<int64_t>(m) * p.ldy + n] = *reinterpret_cast<const uint16_t *>(&h);
-        }
-      }
-    }
-  }
+  swap_epilogue<MPAD, RAW_OUT>(p, tmem_base, tfull, abort_flag, smem, warp, lane, tile, rank, split,
+                               p.s_a);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
