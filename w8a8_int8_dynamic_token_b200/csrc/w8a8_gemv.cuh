@@ -13,7 +13,8 @@
 //      vectors of each row in flight (evict-first loads; the first pair's
 //      loads are issued before step 1 so the prologue hides under them, and
 //      before waiting on the preceding kernel when launched as a programmatic
-//      dependent),
+//      dependent; the warp's next pair is prefetched into L2 by two bulk
+//      prefetches while it works on the current one),
 //      accumulating M int32 dot products with dp4a (exact: every partial sum
 //      is bounded by 127*127*K < 2^31);
 //   3. a warp reduction, then lane m writes
@@ -59,6 +60,14 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *red) {
 #pragma unroll
   for (int w = 0; w < kGemvThreads / 32; ++w) v = max(v, red[w]);
   return v;
+}
+
+// Asks the memory system to bring `bytes` (a multiple of 16) of global memory
+// at `src` (16-byte aligned) into L2; there is no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
+               "r"(bytes)
+               : "memory");
 }
 
 constexpr int kGemvWarps = kGemvThreads / 32;
@@ -188,10 +197,19 @@ __global__ void __launch_bounds__(kGemvThreads, 2) gemv_i8_kernel(const GemvPara
     }
   }
 
-  // ---- 2. stream weight rows, two rows per warp step
+  // ---- 2. stream weight rows, two rows per warp step.  Before working on a
+  // pair, lanes 0 and 1 ask for the warp's next pair of rows to be brought
+  // into L2 (one bulk prefetch per row), so the weight stream from HBM goes
+  // on while the warp computes and reduces; the register loads of the next
+  // pair then come from L2.
   bool loaded = true;  // wv already holds (pi, kb = 0)
   for (; pi < npairs; pi += warps_total) {
     const int n0 = pi * kGemvRows;
+    {
+      const int nn = n0 + warps_total * kGemvRows + lane;
+      if (lane < kGemvRows && nn < p.N)
+        bulk_prefetch_l2(p.wq + static_cast<int64_t>(nn) * K, static_cast<uint32_t>(K));
+    }
     int acc[kGemvRows][MT];
 #pragma unroll
     for (int r = 0; r < kGemvRows; ++r)
