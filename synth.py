@@ -115,6 +115,8 @@ FFN_UP = LayerCase("ffn_up", 4352, 3072, 12288, "studentt", 0)
 FFN_DOWN = LayerCase("ffn_down", 4352, 12288, 3072, "gelu", 0)
 ADALN_M1 = LayerCase("adaln_m1", 1, 3072, 18432, "normal", 0)
 ADALN_M2 = LayerCase("adaln_m2", 2, 3072, 18432, "normal", 0)
+# the same projection for a batch of 16 conditioning vectors
+ADALN_M16 = LayerCase("adaln_m16", 16, 3072, 18432, "normal", 0)
 
 # One DiT block's quantized linears at CFG batch 2 (the conditional and
 # unconditional branches batched: M = 2 x 4352 tokens): the fused q|k|v
@@ -145,4 +147,4 @@ def sweep_cases(ms=SWEEP_M, kns=SWEEP_KN, seeds=SWEEP_SEEDS):
     return out
 
 
-NAMED = {c.name: c for c in (TINY, QKV, FFN_UP, FFN_DOWN, ADALN_M1, ADALN_M2)}
+NAMED = {c.name: c for c in (TINY, QKV, FFN_UP, FFN_DOWN, ADALN_M1, ADALN_M2, ADALN_M16)}

@@ -366,7 +366,7 @@ def _run_layer_sampled(case: synth.LayerCase, check_weights=False):
 
 
 @pytest.mark.parametrize("case", [synth.QKV, synth.FFN_UP, synth.FFN_DOWN, synth.ADALN_M1,
-                                  synth.ADALN_M2], ids=lambda c: c.name)
+                                  synth.ADALN_M2, synth.ADALN_M16], ids=lambda c: c.name)
 def test_full_size_configs(case):
     assert _run_layer_sampled(case, check_weights=True) == 0
 

@@ -24,6 +24,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "w8a8_prefetch.cuh"
 #include "w8a8_ptx.cuh"
 #include "w8a8_quant.cuh"
 
@@ -60,14 +61,6 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *red) {
 #pragma unroll
   for (int w = 0; w < kGemvThreads / 32; ++w) v = max(v, red[w]);
   return v;
-}
-
-// Asks the memory system to bring `bytes` (a multiple of 16) of global memory
-// at `src` (16-byte aligned) into L2; there is no completion to wait for.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)),
-               "r"(bytes)
-               : "memory");
 }
 
 constexpr int kGemvWarps = kGemvThreads / 32;
