@@ -15,12 +15,13 @@
 // shared memory stores, no global workspace), which then runs the epilogue
 //     y[m, n] = bf16_rne( ((float)acc * s_a[m]) * s_w[n] + (float)bias[n] ).
 //
-// Warp roles: warp 0 producer (TMA loads of the Wq box and the q box of each
-// 128-deep k-block into a STAGES-deep ring; the first ring of Wq boxes is
-// issued before the programmatic-dependency wait, since the weights do not
-// depend on the preceding kernel), warp 1 TMEM allocation and the single MMA
-// thread, warps 2..5 the epilogue (one TMEM lane quarter each: lane = weight
-// row n, column = activation row m).  Every wait is bounded.
+// Warp roles: warps 0 and 6 producers (TMA loads of the Wq box and the q box
+// of each 128-deep k-block into a STAGES-deep ring, alternate k-blocks each;
+// the first ring of Wq boxes is issued before the programmatic-dependency
+// wait, since the weights do not depend on the preceding kernel), warp 1 TMEM
+// allocation and the single MMA thread, warps 2..5 the epilogue (one TMEM
+// lane quarter each: lane = weight row n, column = activation row m).  Every
+// wait is bounded.
 #pragma once
 
 #include <cuda.h>
@@ -32,7 +33,8 @@
 
 namespace w8a8 {
 
-constexpr int kSwThreads = 192;  // 6 warps
+constexpr int kSwThreads = 224;  // 7 warps
+constexpr int kSwLoadWarp2 = 6;  // the second load-issuing warp
 constexpr int kSwMaxSplit = 8;   // CTAs of a cluster sharing one tile along K
 
 template <int MPAD>
@@ -53,6 +55,7 @@ struct SwapLayout {
   static constexpr int kSmemBytes = kBarOffset + kBarBytes + 1024;
   static constexpr int kTmemCols = MPAD < 32 ? 32 : MPAD;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kStages % 2 == 0, "the two load threads own alternate stages");
 };
 
 struct SwapParams {
@@ -88,7 +91,7 @@ __device__ __forceinline__ void swap_epilogue(const SwapParams &p, uint32_t tmem
                                               uint64_t *tfull, volatile int *abort_flag,
                                               uint8_t *ring, int warp, int lane, int tile,
                                               int rank, int split, const float *s_a) {
-  const bool epi = warp >= 2;
+  const bool epi = warp >= 2 && warp < 6;
   const int quarter = warp & 3;
   const int row_local = quarter * 32 + lane;          // 0..127 within the tile
   const int n = tile * kBM + row_local;
@@ -205,42 +208,40 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == kSwLoadWarp2) {
+    // ------------------------------------------------------------ producers
+    // Two threads issue the loads, thread u the k-blocks i with i % 2 == u
+    // (so each owns every other stage of the even-sized ring): one thread
+    // waiting on each stage before refilling it sustains about half the TMA
+    // box throughput per SM that two do.
     if (lane == 0) {
+      const int u = warp == 0 ? 0 : 1;
       const int nkb = kb1 - kb0;
-      int prefetched = nkb < S ? nkb : S;
-      for (int i = 0; i < prefetched; ++i) {
+      const int pre = nkb < S ? nkb : S;
+      for (int i = u; i < pre; i += 2) {
         mbar_arrive_expect_tx(&full[i], L::kStageBytes);
         tma_load_2d(&tmap_w, &full[i], smem + i * L::kStageBytes, (kb0 + i) * kBK, tile * kBM);
       }
       grid_dependency_wait();  // q is written by the preceding kernel
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) break;
+      int last = 0;            // one past the last k-block this thread issued
+      for (int i = u; i < nkb; i += 2) {
+        const int stage = i % S;
         uint8_t *sa = smem + stage * L::kStageBytes;
-        if (prefetched > 0) {
-          --prefetched;
-        } else {
+        if (i >= S) {
+          if (!mbar_wait(&empty[stage], static_cast<uint32_t>((i / S) & 1) ^ 1u, abort_flag)) break;
           mbar_arrive_expect_tx(&full[stage], L::kStageBytes);
-          tma_load_2d(&tmap_w, &full[stage], sa, kb * kBK, tile * kBM);
+          tma_load_2d(&tmap_w, &full[stage], sa, (kb0 + i) * kBK, tile * kBM);
         }
-        tma_load_2d(&tmap_q, &full[stage], sa + L::kABytes, kb * kBK, 0);
-        ++issued;
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        tma_load_2d(&tmap_q, &full[stage], sa + L::kABytes, (kb0 + i) * kBK, 0);
+        last = i + 1;
       }
-      grid_dependents_launch();
-      // every load issued has been consumed by an MMA (or, after an abort,
-      // is waited for here) before the ring is reused or the CTA leaves
-      const uint32_t n = issued < static_cast<uint32_t>(S) ? issued : S;
-      for (uint32_t i = issued - n; i < issued; ++i) {
+      if (u == 0) grid_dependents_launch();
+      // every load this thread issued has been consumed by an MMA (or, after
+      // an abort, is waited for here) before the CTA leaves
+      for (int i = (last > S ? last - S : 0); i < last; ++i) {
+        if ((i & 1) != u) continue;
         volatile int never = 0;
-        mbar_wait(&full[i % S], (i / S) & 1u, &never);
+        mbar_wait(&full[i % S], static_cast<uint32_t>((i / S) & 1), &never);
       }
     }
   } else if (warp == 1) {
