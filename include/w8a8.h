@@ -250,6 +250,13 @@ W8A8_API int w8a8_linear_fused_ex(const void *x_bf16, int64_t M, int64_t K, int6
  * y_dev [M,N] dense are caller-owned device staging buffers; Wq, s_w, bias and
  * workspace are device pointers as in w8a8_linear_fused.  The call returns
  * after enqueueing; synchronize `stream` before reading y_host.
+ * The rows go in up to 8 chunks (at least 256 rows each): chunk c is copied
+ * in on `stream`, computed on an internal stream of the library and copied
+ * out on a second internal one, so that the two copy directions and the
+ * layer overlap; the internal streams fork from and join back into `stream`
+ * through events (the call may be captured in a CUDA graph).  The result is
+ * identical to one layer call over all rows.  Calls on one device take a
+ * library mutex while they enqueue.
  */
 W8A8_API int w8a8_linear_fused_host(const void *x_host, int64_t M, int64_t K,
                            const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null,

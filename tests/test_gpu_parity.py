@@ -404,21 +404,57 @@ def test_sweep_point(case):
 
 # ----------------------------------------------------------------- host buffers
 
-@pytest.mark.parametrize("M,N,K", [(64, 128, 256), (300, 520, 3072), (2, 1032, 3072)])
+# (M, N, K): one chunk; 256 + 44 rows; two rows; six chunks of 384 rows
+@pytest.mark.parametrize("M,N,K", [(64, 128, 256), (300, 520, 3072), (2, 1032, 3072),
+                                   (2304, 1032, 1024)])
 def test_linear_fused_host_buffers(M, N, K):
+    """Host buffers in and out, the rows in chunks whose copies and layer
+    calls run on three streams: y against the oracle in full.  The staging
+    buffers start out holding other values, so a chunk computed before its
+    copy in, or copied out before its layer, shows."""
     x, w, b = synth.make_x(M, K, "studentt", 4), synth.make_w(N, K, 4), synth.make_bias(N, 4)
     wq_ref, sw_ref = oracle.quantize_weights(w)
     ref = oracle.linear(x, wq_ref, sw_ref, b)
     x_host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
     y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
-    y_dev = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    x_dev = torch.full((M, K), 3.0, dtype=torch.bfloat16, device="cuda")
+    y_dev = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
     nws = w8a8.workspace_size(M, N, K)
     ws = torch.empty((max(nws, 1),), dtype=torch.uint8, device="cuda")
     w8a8.linear_fused_host(x_host, torch.from_numpy(wq_ref).cuda(),
                            torch.from_numpy(sw_ref).cuda(), to_dev(b), y_host, x_dev, y_dev, ws)
     torch.cuda.current_stream().synchronize()
     assert check_y(bits_of(y_host), ref["y"], ref["y32"], "host buffers") == 0
+
+
+def test_linear_fused_host_buffers_in_a_cuda_graph():
+    """The chunked host-buffer call captured once (its internal streams fork
+    from and join back into the capturing stream) and replayed on new host
+    inputs: each replay's y_host matches the oracle for that input."""
+    M, N, K = 1100, 264, 512
+    w, b = synth.make_w(N, K, 6), synth.make_bias(N, 6)
+    wq_ref, sw_ref = oracle.quantize_weights(w)
+    Wq, s_w, bd = torch.from_numpy(wq_ref).cuda(), torch.from_numpy(sw_ref).cuda(), to_dev(b)
+    x_host = torch.empty((M, K), dtype=torch.bfloat16).pin_memory()
+    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    y_dev = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((w8a8.workspace_size(M, N, K),), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            w8a8.linear_fused_host(x_host, Wq, s_w, bd, y_host, x_dev, y_dev, ws, stream=s)
+    torch.cuda.synchronize()
+    for seed in (7, 8):
+        x = synth.make_x(M, K, "normal", seed)
+        x_host.copy_(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16))
+        g.replay()
+        torch.cuda.synchronize()
+        ref = oracle.linear(x, wq_ref, sw_ref, b)
+        assert check_y(bits_of(y_host), ref["y"], ref["y32"], f"graph replay {seed}") == 0
+    del g
 
 
 # ----------------------------------------------------------------- failure detection

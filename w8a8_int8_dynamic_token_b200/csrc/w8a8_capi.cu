@@ -1204,6 +1204,42 @@ int w8a8_linear_fused_noalloc(const void *x, int64_t M, int64_t K, int64_t ldx, 
                            kNoAllocScratchBytes, stream);
 }
 
+// The end-to-end call splits the rows into up to kHostChunks chunks: chunk
+// c's copy in (on the caller's stream), its layer (on an internal stream) and
+// its copy out (on another) overlap the other chunks' work, so the copies in
+// and out -- PCIe carries both directions at once -- run side by side with
+// the layer.  Every output depends on its own row only, so the result is the
+// same as one call over all rows.  The internal streams and events are made
+// once per device and reused; a mutex orders the calls that enqueue on them.
+constexpr int kHostChunks = 8;
+constexpr int64_t kHostChunkMinRows = 256;
+
+struct HostPipe {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t compute = nullptr, d2h = nullptr;
+  cudaEvent_t fork = nullptr, done = nullptr;
+  cudaEvent_t in[kHostChunks] = {}, out[kHostChunks] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+
+int host_pipe_ready(HostPipe &hp) {
+  if (hp.ready) return W8A8_OK;
+  bool ok = cudaStreamCreateWithFlags(&hp.compute, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&hp.fork, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming) == cudaSuccess;
+  for (int c = 0; ok && c < kHostChunks; ++c)
+    ok = cudaEventCreateWithFlags(&hp.in[c], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&hp.out[c], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    return W8A8_ERR_CUDA;
+  }
+  hp.ready = true;
+  return W8A8_OK;
+}
+
 int w8a8_linear_fused_host(const void *x_host, int64_t M, int64_t K, const int8_t *Wq,
                            const float *s_w, const void *bias, int64_t N, void *y_host,
                            void *x_dev, void *y_dev, void *workspace, size_t ws_bytes,
@@ -1217,20 +1253,59 @@ int w8a8_linear_fused_host(const void *x_host, int64_t M, int64_t K, const int8_
   const DeviceInfo *d = nullptr;
   st = query_device(&d);
   if (st != W8A8_OK) return st;
-  if (cudaMemcpyAsync(x_dev, x_host, static_cast<size_t>(M * K) * 2, cudaMemcpyHostToDevice,
-                      stream) != cudaSuccess) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return W8A8_ERR_CUDA;
   }
-  st = w8a8_linear_fused(x_dev, M, K, K, Wq, s_w, bias, N, y_dev, N, nullptr, nullptr, workspace,
-                         ws_bytes, stream_);
+  HostPipe &hp = g_pipe[dev];
+  std::lock_guard<std::mutex> lock(hp.mu);
+  st = host_pipe_ready(hp);
   if (st != W8A8_OK) return st;
-  if (cudaMemcpyAsync(y_host, y_dev, static_cast<size_t>(M * N) * 2, cudaMemcpyDeviceToHost,
-                      stream) != cudaSuccess) {
+  // chunks of at least kHostChunkMinRows rows, a multiple of 128
+  int64_t rows_per = cdiv(M, kHostChunks);
+  if (rows_per < kHostChunkMinRows) rows_per = kHostChunkMinRows;
+  rows_per = cdiv(rows_per, 128) * 128;
+  const int64_t nch = cdiv(M, rows_per);  // <= kHostChunks
+  const uint8_t *xh = static_cast<const uint8_t *>(x_host);
+  uint8_t *yh = static_cast<uint8_t *>(y_host);
+  uint8_t *xd = static_cast<uint8_t *>(x_dev);
+  uint8_t *yd = static_cast<uint8_t *>(y_dev);
+  // fork: the internal streams start after the work already on `stream`
+  bool cuda_ok = cudaEventRecord(hp.fork, stream) == cudaSuccess &&
+                 cudaStreamWaitEvent(hp.compute, hp.fork, 0) == cudaSuccess &&
+                 cudaStreamWaitEvent(hp.d2h, hp.fork, 0) == cudaSuccess;
+  st = W8A8_OK;
+  for (int64_t c = 0; cuda_ok && st == W8A8_OK && c < nch; ++c) {
+    const int64_t r0 = c * rows_per;
+    const int64_t rows = M - r0 < rows_per ? M - r0 : rows_per;
+    const size_t xoff = static_cast<size_t>(r0 * K) * 2, xbytes = static_cast<size_t>(rows * K) * 2;
+    const size_t yoff = static_cast<size_t>(r0 * N) * 2, ybytes = static_cast<size_t>(rows * N) * 2;
+    cuda_ok = cudaMemcpyAsync(xd + xoff, xh + xoff, xbytes, cudaMemcpyHostToDevice, stream) ==
+                  cudaSuccess &&
+              cudaEventRecord(hp.in[c], stream) == cudaSuccess &&
+              cudaStreamWaitEvent(hp.compute, hp.in[c], 0) == cudaSuccess;
+    if (!cuda_ok) break;
+    st = w8a8_linear_fused(xd + xoff, rows, K, K, Wq, s_w, bias, N, yd + yoff, N, nullptr, nullptr,
+                           workspace, ws_bytes, reinterpret_cast<w8a8_stream_t>(hp.compute));
+    if (st != W8A8_OK) break;
+    cuda_ok = cudaEventRecord(hp.out[c], hp.compute) == cudaSuccess &&
+              cudaStreamWaitEvent(hp.d2h, hp.out[c], 0) == cudaSuccess &&
+              cudaMemcpyAsync(yh + yoff, yd + yoff, ybytes, cudaMemcpyDeviceToHost, hp.d2h) ==
+                  cudaSuccess;
+  }
+  // join: `stream` continues once the last copy out (and, through the
+  // events, every chunk's layer) is done -- also after an error, so that
+  // the streams stay ordered
+  const bool joined = cudaEventRecord(hp.out[0], hp.compute) == cudaSuccess &&
+                      cudaStreamWaitEvent(hp.d2h, hp.out[0], 0) == cudaSuccess &&
+                      cudaEventRecord(hp.done, hp.d2h) == cudaSuccess &&
+                      cudaStreamWaitEvent(stream, hp.done, 0) == cudaSuccess;
+  if (!cuda_ok || !joined) {
     cudaGetLastError();
     return W8A8_ERR_CUDA;
   }
-  return W8A8_OK;
+  return st;
 }
 
 int w8a16_linear(const void *x, int64_t M, int64_t K, int64_t ldx, const int8_t *Wq,
