@@ -480,6 +480,40 @@ def test_errors_are_returned_not_raised_in_c():
 
 # ----------------------------------------------------------------- chained calls
 
+@pytest.mark.parametrize("M,N,K", [(4352, 9216, 3072), (64, 9216, 3072), (3, 18432, 3072),
+                                   (16, 18432, 3072)])
+def test_layer_right_after_quantize_weights(M, N, K):
+    """Weight quantization into a buffer holding other values, then at once
+    on the same stream a layer on precomputed q reading that Wq (the pair
+    GEMM, the one-CTA GEMM, the GEMV, the tensor-core small-M kernel: each
+    prefetches weights before its dependency wait).  The weight kernel must
+    release its dependents only when it has completed, so the layer sees the
+    finished weights: y must equal the layer run after a full synchronize."""
+    dev = torch.device("cuda")
+    W = to_dev(synth.make_w(N, K, 11))
+    q, s_a = w8a8.quant_act(to_dev(synth.make_x(M, K, "normal", 11)))
+    Wq, s_w = torch.empty((N, K), dtype=torch.int8, device=dev), torch.empty(N, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((max(1, w8a8.workspace_size(M, N, K)),), dtype=torch.uint8, device=dev)
+    s = B._stream()
+
+    def run():
+        assert B.w8a8_quantize_weights(B._ptr(W), N, K, K, B._ptr(Wq), B._ptr(s_w), s) == 0
+        assert B.w8a8_linear(B._ptr(q), B._ptr(s_a), M, K, B._ptr(Wq), B._ptr(s_w), None, N,
+                             B._ptr(y), N, None, B._ptr(ws), ws.numel(), s) == 0
+
+    run()
+    torch.cuda.synchronize()
+    ref = y.clone()
+    for fill in (7, -100, 0):
+        Wq.fill_(fill)
+        s_w.fill_(float(fill))
+        y.fill_(float("nan"))
+        run()
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), f"fill {fill}"
+
+
 def test_chained_layers_share_buffers_under_dependent_launch():
     """Consecutive layer calls are launched as programmatic dependents: each
     kernel starts before the previous one finishes and waits for it before

@@ -537,8 +537,11 @@ void quant_bulk_shape(int64_t K, int *group_warps, int *slots) {
   *slots = static_cast<int>(sl);
 }
 
+// release_early: let the kernel that follows be launched as soon as this one
+// starts (activations; never for weights, see quant_rows_kernel).
 int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q, float *s,
-                 cudaStream_t stream) {
+                 bool release_early, cudaStream_t stream) {
+  const int rel = release_early ? 1 : 0;
   const uint16_t *xp = static_cast<const uint16_t *>(x);
   if (rows > INT32_MAX / 2) return W8A8_ERR_UNSUPPORTED_SHAPE;
   const DeviceInfo *d = nullptr;
@@ -561,7 +564,7 @@ int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q,
     if (grid > d->sms) grid = d->sms;
     return launch_ex(true, quant_rows_bulk_kernel, dim3(static_cast<unsigned>(grid)),
                      dim3(kQuantBulkWarps * 32), static_cast<size_t>(smem), stream, xp,
-                     static_cast<int>(rows), static_cast<int>(K), ldx, q, s, gw, slots);
+                     static_cast<int>(rows), static_cast<int>(K), ldx, q, s, gw, slots, rel);
   }
   // G threads per row (32 .. 256), each holding V <= kQuantMaxV vectors of
   // 8 bf16 in registers, and G widened until the rows fill the SMs (or one
@@ -575,14 +578,14 @@ int launch_quant(const void *x, int64_t rows, int64_t K, int64_t ldx, int8_t *q,
   }
   if (V > kQuantMaxV) {  // rows longer than 256 x 12 x 8 = 24576 elements
     return launch_ex(true, quant_rows_long_kernel, dim3(static_cast<unsigned>(rows)), dim3(256), 0,
-                     stream, xp, K, ldx, q, s);
+                     stream, xp, K, ldx, q, s, rel);
   }
   const int rows_per_block = 256 / G;
   const int64_t grid = cdiv(rows, rows_per_block);
   const int r32 = static_cast<int>(rows), k32 = static_cast<int>(K);
 #define W8A8_QUANT_CASE(VV)                                                                \
   return launch_ex(true, quant_rows_kernel<VV>, dim3(static_cast<unsigned>(grid)), dim3(256), \
-                   0, stream, xp, r32, k32, ldx, q, s, G)
+                   0, stream, xp, r32, k32, ldx, q, s, G, rel)
   switch (V) {
     case 1: W8A8_QUANT_CASE(1);
     case 2: W8A8_QUANT_CASE(2);
@@ -1011,7 +1014,7 @@ int w8a8_quantize_weights(const void *W, int64_t N, int64_t K, int64_t ldw, int8
   const DeviceInfo *d = nullptr;
   st = query_device(&d);
   if (st != W8A8_OK) return st;
-  return launch_quant(W, N, K, ldw, Wq, s_w, reinterpret_cast<cudaStream_t>(stream));
+  return launch_quant(W, N, K, ldw, Wq, s_w, false, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_unpack_int32_weights(const int32_t *packed, int64_t N, int64_t K, int8_t *Wq,
@@ -1041,7 +1044,7 @@ int w8a8_quant_act(const void *x, int64_t M, int64_t K, int64_t ldx, int8_t *q, 
   const DeviceInfo *d = nullptr;
   st = query_device(&d);
   if (st != W8A8_OK) return st;
-  return launch_quant(x, M, K, ldx, q, s_a, reinterpret_cast<cudaStream_t>(stream));
+  return launch_quant(x, M, K, ldx, q, s_a, true, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8a8_select(int64_t M, int64_t N, int64_t K, int32_t num_sms, int variant,
@@ -1178,7 +1181,7 @@ int w8a8_linear_fused_ex(const void *x, int64_t M, int64_t K, int64_t ldx, const
     st = clear_counters(split.counters, split.counters ? split_counter_bytes(plan) : 0, stream);
     if (st != W8A8_OK) return st;
   }
-  st = launch_quant(x, M, K, ldx, q, s_a, stream);
+  st = launch_quant(x, M, K, ldx, q, s_a, true, stream);
   if (st != W8A8_OK) return st;
   return linear_impl(q, s_a, M, K, Wq, s_w, bias, N, y, ldy, nullptr, plan.variant, split_ws,
                      split_bytes, true, stream);

@@ -174,14 +174,15 @@ __device__ __forceinline__ void quant_row_by_warp(const uint16_t *__restrict__ x
 __global__ void __launch_bounds__(256) quant_rows_long_kernel(const uint16_t *__restrict__ x,
                                                               int64_t K, int64_t ldx,
                                                               int8_t *__restrict__ q,
-                                                              float *__restrict__ s) {
+                                                              float *__restrict__ s,
+                                                              int release_early) {
   __shared__ uint32_t red[8];
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x;
   const int64_t nvec = K >> 3;
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * ldx);
-  grid_dependency_wait();  // see quant_rows_kernel
-  grid_dependents_launch();
+  if (release_early) grid_dependents_launch();  // see quant_rows_kernel
+  grid_dependency_wait();
   float m = 0.0f;
   for (int64_t vi = tid; vi < nvec; vi += 256) m = absmax_vec8(__ldg(xr + vi), m);
   uint32_t mb = warp_max_u32(__float_as_uint(m), 32);
@@ -315,7 +316,7 @@ __device__ __forceinline__ void quant_row_from_smem(const uint4 *xs, int K, int8
 __global__ void __launch_bounds__(kQuantBulkWarps * 32, 1)
     quant_rows_bulk_kernel(const uint16_t *__restrict__ x, int rows, int K, int64_t ldx,
                            int8_t *__restrict__ q, float *__restrict__ s, int group_warps,
-                           int slots) {
+                           int slots, int release_early) {
   extern __shared__ __align__(128) uint8_t quant_slots[];
   __shared__ uint64_t bars[kQuantBulkWarps * kQuantBulkMaxSlots];
   __shared__ uint32_t red[kQuantBulkWarps];
@@ -337,8 +338,8 @@ __global__ void __launch_bounds__(kQuantBulkWarps * 32, 1)
     for (int j = 0; j < slots; ++j) mbar_init(&bar[j], 1);
   fence_mbarrier_init();
   __syncthreads();
-  // launched as a programmatic dependent: x may come from the preceding
-  // kernel, and q / s may still be read by it
+  // see quant_rows_kernel
+  if (release_early) grid_dependents_launch();
   grid_dependency_wait();
   int issued = 0;
   if (leader) {
@@ -348,7 +349,6 @@ __global__ void __launch_bounds__(kQuantBulkWarps * 32, 1)
       bulk_load_g2s(mine + issued * row_bytes, x + row * ldx, row_bytes, &bar[issued]);
     }
   }
-  grid_dependents_launch();  // the GEMM that follows may start its prologue
   const int nvec = K >> 3;
   const int gthreads = G * 32;
   const int t = gw * 32 + lane;   // thread index within the group
@@ -424,7 +424,8 @@ template <int V>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t *__restrict__ x,
                                                          int rows, int K, int64_t ldx,
                                                          int8_t *__restrict__ q,
-                                                         float *__restrict__ s, int G) {
+                                                         float *__restrict__ s, int G,
+                                                         int release_early) {
   __shared__ uint32_t red[8];
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -436,8 +437,15 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t *__restr
   const int nvec = K >> 3;
 
   const uint4 *xr = reinterpret_cast<const uint4 *>(x + (row_ok ? row : 0) * ldx);
-  // launched as a programmatic dependent: x may come from the preceding
-  // kernel, and q / s may still be read by it -- wait before either
+  // Launched as a programmatic dependent: x may come from the preceding
+  // kernel, and q / s may still be read by it -- wait before either.  With
+  // release_early (activations), the kernel that follows may be launched at
+  // once: the library's GEMM, GEMV and small-M kernels read only the weights
+  // before their own dependency wait, which completes after this kernel (and,
+  // through this kernel's wait, the one before it).  Without (weights: the
+  // kernel that follows prefetches the very Wq written here), dependents
+  // start only when this grid has completed.
+  if (release_early) grid_dependents_launch();
   grid_dependency_wait();
   uint4 v[V];
 #pragma unroll
@@ -445,7 +453,6 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t *__restr
     const int vi = t + j * G;
     v[j] = (row_ok && vi < nvec) ? __ldcs(xr + vi) : make_uint4(0u, 0u, 0u, 0u);
   }
-  grid_dependents_launch();  // the GEMM that follows may start its prologue
   float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
   for (int j = 0; j < V; ++j) {
