@@ -836,8 +836,11 @@ def test_quantization_fused_into_pair_launch_replayed_in_a_cuda_graph():
 
 # ----------------------------------------------------------------- W8A16 (weight-only)
 
+# ragged N (520, 1032, 264, 4104, 9000), ragged M and K tails (400, 2064 by
+# 16 below a k-block), one tile to many rounds of tiles
 W8A16_CASES = [(64, 128, 256, True), (300, 520, 400, True), (129, 1032, 3072, False),
-               (17, 264, 12288, True), (4352, 9216, 3072, True)]
+               (17, 264, 12288, True), (4352, 9216, 3072, True), (1000, 4104, 1024, True),
+               (2000, 9000, 400, False)]
 
 
 @pytest.mark.parametrize("M,N,K,bias", W8A16_CASES)
