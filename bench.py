@@ -581,20 +581,11 @@ def run_ours(args):
     gclk = gsampler.summary()
     layer.i = 0
     tq = timed(layer.quant_step, gsteps, warmup, dist, graph=True) / gsteps
-    gload = None
     if not small:
-        # the burst peaks first (before the sustained run below heats the part)
+        # the burst peaks (the sustained GEMM run, which heats the part into
+        # the power cap, comes last of all)
         i8 = measure_i8_peak(dev, dist)
         int_mm = measure_int_mm(dev, dist) if world == 1 else None
-        # the SM clock the GEMM holds under sustained load (the power cap can
-        # hold it below the clock of a short burst): about 0.4 s of graph
-        # replays of the same GEMM steps, sampled every 2 ms
-        layer.i = 0
-        lsampler = ClockSampler(dev.index if dev.index is not None else 0)
-        reps = max(2, int(0.4 / max(tg * gsteps, 1e-6)))
-        tl = timed(layer.gemm_step, gsteps, 0, dist, lsampler, graph=True, replays=reps)
-        gload = dict(lsampler.summary(), us_per_launch=round(tl / (reps * gsteps) * 1e6, 2),
-                     seconds=round(tl, 3))
     if small:
         if layer.one_launch:
             # the GEMV quantizing its rows itself: the kernel is the layer
@@ -641,17 +632,6 @@ def run_ours(args):
             roofline["torch_int_mm_8192"] = int_mm
             if int_mm.get("tops"):
                 roofline["frac_of_torch_int_mm_8192"] = round(achieved / int_mm["tops"], 4)
-        if gload is not None:
-            roofline["gemm_sustained_0p4s"] = gload
-        if gload and gload.get("sm_mhz") and i8.get("ops_per_clk_per_sm"):
-            # the measured per-clock rate at the clock the GEMM holds under
-            # sustained load, against the GEMM's rate in that same run
-            clock_peak = sms * i8["ops_per_clk_per_sm"] * gload["sm_mhz"] * 1e6 / 1e12
-            sustained = ops / (gload["us_per_launch"] * 1e-6) / 1e12
-            roofline["frac_of_peak_at_gemm_clock"] = round(sustained / clock_peak, 4)
-            roofline["peak_at_gemm_clock_tops"] = round(clock_peak, 1)
-            roofline["gemm_clock_basis"] = ("median SM clock of the 0.4 s sustained run; its "
-                                            "rate against the measured per-clock peak")
     quant_bytes = 3 * M * K + 4 * M
     layer.i = 0
     t_single = single_launch_us(layer.step)
@@ -675,13 +655,35 @@ def run_ours(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(te / esteps * 1e3, 3)}
     launches = layer.launches_per_step
-    del layer
-    torch.cuda.empty_cache()
 
     components = {}
     if not args.no_extras and world == 1:
         components = extra_components(args, dev, dist, peaks, world,
                                       roofline.get("peak") if not small else None)
+
+    if not small:
+        # the SM clock the GEMM holds under sustained load (the power cap can
+        # hold it below the clock of a short burst): about 0.4 s of graph
+        # replays of the same GEMM steps, sampled every 2 ms -- run last, so
+        # that the heat it leaves throttles no other measurement
+        layer.i = 0
+        lsampler = ClockSampler(dev.index if dev.index is not None else 0)
+        reps = max(2, int(0.4 / max(tg * gsteps, 1e-6)))
+        tl = timed(layer.gemm_step, gsteps, 0, dist, lsampler, graph=True, replays=reps)
+        gload = dict(lsampler.summary(), us_per_launch=round(tl / (reps * gsteps) * 1e6, 2),
+                     seconds=round(tl, 3))
+        roofline["gemm_sustained_0p4s"] = gload
+        if gload.get("sm_mhz") and i8.get("ops_per_clk_per_sm"):
+            # the measured per-clock rate at the clock the GEMM holds under
+            # sustained load, against the GEMM's rate in that same run
+            clock_peak = sms * i8["ops_per_clk_per_sm"] * gload["sm_mhz"] * 1e6 / 1e12
+            sustained = ops / (gload["us_per_launch"] * 1e-6) / 1e12
+            roofline["frac_of_peak_at_gemm_clock"] = round(sustained / clock_peak, 4)
+            roofline["peak_at_gemm_clock_tops"] = round(clock_peak, 1)
+            roofline["gemm_clock_basis"] = ("median SM clock of the 0.4 s sustained run; its "
+                                            "rate against the measured per-clock peak")
+    del layer
+    torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
