@@ -304,6 +304,10 @@ def timed(fn, steps: int, warmup: int, dist=None, sampler=None, graph=False, rep
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ctx = sampler if sampler is not None else _Null()
     with ctx:
+        # a ~0.1 ms spin ahead of the start event keeps the device busy while
+        # the host enqueues the first steps, so the timed region holds the K
+        # steps back to back and not the host's latency to the first launch
+        torch.cuda._sleep(200_000)
         e0.record(stream)
         for _ in range(steps_run):
             fn()
