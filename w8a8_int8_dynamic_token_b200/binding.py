@@ -214,6 +214,8 @@ def _ptr(t):
 
 
 def _stream(stream=None):
+    if isinstance(stream, int):  # a raw handle (see _OnCurrent)
+        return ctypes.c_void_p(stream)
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
 
@@ -251,14 +253,37 @@ def _on_one_device(**tensors):
     return dev
 
 
-@contextlib.contextmanager
+class _OnCurrent:
+    """The common case of _launching: the tensors' device is already current
+    and no stream is given, so nothing needs switching; yields that device's
+    current stream as a raw handle."""
+    __slots__ = ("handle",)
+
+    def __init__(self, handle):
+        self.handle = handle
+
+    def __enter__(self):
+        return self.handle
+
+    def __exit__(self, *exc):
+        return False
+
+
 def _launching(dev, stream=None):
     """Run a call on the tensors' device: the library reads the current device
     (its properties, and the allocation-free scratch), so that device is made
     current.  The call is enqueued on `stream`, or on that device's current
     stream; tensors allocated inside belong to that stream, so the caching
     allocator never hands their memory to other work while the call may still
-    use it."""
+    use it.  When the device is current already and no stream is given,
+    nothing is switched (a few microseconds of host time per call less)."""
+    if stream is None and dev.index == torch.cuda.current_device():
+        return _OnCurrent(torch._C._cuda_getCurrentRawStream(dev.index))
+    return _switching(dev, stream)
+
+
+@contextlib.contextmanager
+def _switching(dev, stream):
     with torch.cuda.device(dev):
         if stream is None:
             yield torch.cuda.current_stream()

@@ -388,7 +388,53 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
 }
 
 // int8 matrix [rows, K] dense, box = 128 (K) x box_rows, 128-byte swizzle.
+// Tensor maps encoded earlier on this thread, keyed by everything that goes
+// into them (which map form, base address, extents, row stride, box rows): a
+// map holds addresses and shapes only, so a hit is the map a new encoding
+// would produce.  Encoding costs host time on every layer call otherwise.
+struct MapKey {
+  int kind;
+  const void *base;
+  int64_t rows, cols, ld;
+  int box;
+  bool operator==(const MapKey &o) const {
+    return kind == o.kind && base == o.base && rows == o.rows && cols == o.cols && ld == o.ld &&
+           box == o.box;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  bool valid;
+  CUtensorMap map;
+};
+constexpr int kMapCacheSize = 64;
+thread_local MapEntry t_map_cache[kMapCacheSize];
+
+MapEntry &map_slot(const MapKey &k) {
+  uint64_t h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+  h ^= static_cast<uint64_t>(k.kind) * 0xC2B2AE3D27D4EB4Full + static_cast<uint64_t>(k.rows) * 31u +
+       static_cast<uint64_t>(k.cols) * 131u + static_cast<uint64_t>(k.ld) * 7u +
+       static_cast<uint64_t>(k.box);
+  return t_map_cache[(h >> 32) % kMapCacheSize];
+}
+
+bool map_lookup(const MapKey &k, CUtensorMap *out) {
+  const MapEntry &e = map_slot(k);
+  if (!e.valid || !(e.key == k)) return false;
+  *out = e.map;
+  return true;
+}
+
+void map_store(const MapKey &k, const CUtensorMap &m) {
+  MapEntry &e = map_slot(k);
+  e.key = k;
+  e.map = m;
+  e.valid = true;
+}
+
 int encode_i8_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, int box_rows) {
+  const MapKey key{1, base, rows, K, K, box_rows};
+  if (map_lookup(key, map)) return W8A8_OK;
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
   if (enc == nullptr) return W8A8_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
@@ -398,13 +444,17 @@ int encode_i8_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K, i
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+  if (r != CUDA_SUCCESS) return W8A8_ERR_CUDA;
+  map_store(key, *map);
+  return W8A8_OK;
 }
 
 // bf16 matrix [rows, cols] with row stride ld elements, box 64 (cols) x
 // box_rows, 128-byte swizzle (the W8A16 GEMM's activation operand).
 int encode_bf16_load_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols,
                          int64_t ld, int box_rows) {
+  const MapKey key{2, base, rows, cols, ld, box_rows};
+  if (map_lookup(key, map)) return W8A8_OK;
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
   if (enc == nullptr) return W8A8_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -414,7 +464,9 @@ int encode_bf16_load_map(CUtensorMap *map, const void *base, int64_t rows, int64
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+  if (r != CUDA_SUCCESS) return W8A8_ERR_CUDA;
+  map_store(key, *map);
+  return W8A8_OK;
 }
 
 // int8 matrix [rows, K] dense, box 64 (K) x box_rows, 64-byte swizzle (the
@@ -422,6 +474,8 @@ int encode_bf16_load_map(CUtensorMap *map, const void *base, int64_t rows, int64
 // 16-byte chunks without bank conflicts).
 int encode_i8_sw64_map(CUtensorMap *map, const void *base, int64_t rows, int64_t K,
                        int box_rows) {
+  const MapKey key{3, base, rows, K, K, box_rows};
+  if (map_lookup(key, map)) return W8A8_OK;
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
   if (enc == nullptr) return W8A8_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
@@ -431,13 +485,17 @@ int encode_i8_sw64_map(CUtensorMap *map, const void *base, int64_t rows, int64_t
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+  if (r != CUDA_SUCCESS) return W8A8_ERR_CUDA;
+  map_store(key, *map);
+  return W8A8_OK;
 }
 
 // bf16 matrix [rows, cols] with row stride ld elements, box 32 x 32, 64-byte
 // swizzle (the epilogue's staging layout).
 int encode_bf16_store_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols,
                           int64_t ld) {
+  const MapKey key{4, base, rows, cols, ld, 0};
+  if (map_lookup(key, map)) return W8A8_OK;
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encoder();
   if (enc == nullptr) return W8A8_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -447,7 +505,9 @@ int encode_bf16_store_map(CUtensorMap *map, const void *base, int64_t rows, int6
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? W8A8_OK : W8A8_ERR_CUDA;
+  if (r != CUDA_SUCCESS) return W8A8_ERR_CUDA;
+  map_store(key, *map);
+  return W8A8_OK;
 }
 
 // ---------------------------------------------------------------- launches
