@@ -44,6 +44,12 @@
  *  - Inputs must be finite: NaN or Inf in x or W is outside the contract.
  *  - Calls on different streams are independent and thread-safe; calls that
  *    share a workspace must be ordered by the caller.
+ *  - State the library keeps: the device properties read at first use; a
+ *    per-thread cache of encoded tensor maps (host memory, keyed by every
+ *    value encoded into a map, so a hit equals a fresh encoding); two
+ *    streams and their events per device for w8a8_linear_fused_host, made at
+ *    its first call and used under a mutex; the static scratch of
+ *    w8a8_linear_fused_noalloc.
  */
 #ifndef W8A8_H
 #define W8A8_H
