@@ -108,9 +108,9 @@ def test_selector_small_m_goes_to_gemv():
     for M in (1, 2, 3):
         p = w8a8.select(M, N, K)
         assert p["variant_name"] == "gemv" and p["quant_in_gemm_launch"] == int(M <= 2)
-    for M in (4, 5, lim):
+    for M in (4, 5, lim, lim + 1, 20):
         assert w8a8.select(M, N, K)["variant_name"] == "gemv_tc"
-    assert w8a8.select(lim + 1, N, K)["variant_name"].startswith("gemm")
+    assert w8a8.select(21, N, K)["variant_name"].startswith("gemm")
     assert w8a8.select(lim, N, K, variant=B.VARIANT_GEMV)["variant_name"] == "gemv"
     assert w8a8.workspace_size(1, N, K) == 0
     assert w8a8.workspace_size(3, N, K) >= 3 * K + 3 * 4   # q and s_a for the quantization kernel
@@ -144,9 +144,11 @@ def test_selector_gemm_plans():
     # tiny output: few tiles, grid = tiles
     p = w8a8.select(64, 128, 256)
     assert p["grid"] == p["num_tiles"] <= 2
-    # GEMV would need more than 227 KB of shared memory: falls back to GEMM
+    # too deep for the GEMV's shared-memory rows: the tensor-core small-M
+    # variant to 32 rows, the GEMM above
     assert w8a8.select(16, 64, 16384)["variant_name"] == "gemv_tc"
-    assert w8a8.select(17, 64, 16384)["variant_name"].startswith("gemm")
+    assert w8a8.select(32, 64, 16384)["variant_name"] == "gemv_tc"
+    assert w8a8.select(33, 64, 16384)["variant_name"].startswith("gemm")
     # forced variants
     assert w8a8.select(1, 64, 256, variant=B.VARIANT_GEMM_BN128)["tile_n"] == 128
     with pytest.raises(w8a8.W8A8Error):
@@ -261,7 +263,18 @@ def test_pair_k_split_plans():
     assert n >= 8704 * 12288 + 4 * 8704 + (112 + 73) * 256 * 1024
 
 
-@pytest.mark.parametrize("M", [17, 100, 4352, 16384])
+def test_selector_at_17_rows_follows_the_measured_crossovers():
+    # 17 rows, the first above torch._int_mm's limit: the tensor-core small-M
+    # variant on weights at least 9216 wide or 8192 deep, the GEMM otherwise
+    assert w8a8.select(17, 9216, 3072)["variant_name"] == "gemv_tc"
+    assert w8a8.select(17, 12288, 3072)["variant_name"] == "gemv_tc"
+    assert w8a8.select(17, 3072, 12288)["variant_name"] == "gemv_tc"
+    assert w8a8.select(17, 6144, 3072)["variant_name"].startswith("gemm")
+    assert w8a8.select(17, 3072, 3072)["variant_name"].startswith("gemm")
+    assert w8a8.select(24, 9216, 3072)["variant_name"].startswith("gemm")
+
+
+@pytest.mark.parametrize("M", [33, 100, 4352, 16384])
 @pytest.mark.parametrize("KN", [(3072, 9216), (3072, 3072), (3072, 12288), (12288, 3072)])
 def test_selector_is_total_and_consistent(M, KN):
     K, N = KN
@@ -307,7 +320,9 @@ def test_selector_plans_are_valid_for_random_shapes(M, n8, k16):
         return
     tm, tn, tiles = p["tile_m"], p["tile_n"], p["num_tiles"]
     if v == "gemv_tc":
-        assert 4 <= M <= 16 and (N >= 6144 or K >= 8192)
+        assert 4 <= M <= 32
+        assert ((M <= 16 and (N >= 6144 or K >= 8192)) or (M <= 20 and N >= 9216)
+                or K >= 8192)
         assert tm == 128 and tn == 16 and tiles == _cdiv(N, 128)
         ks = p["k_split"]
         assert 1 <= ks <= 8 and ks <= _cdiv(K, 128) and p["grid"] == tiles * ks

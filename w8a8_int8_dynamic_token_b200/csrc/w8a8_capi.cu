@@ -131,11 +131,17 @@ inline bool gemv_quantizes_itself(int64_t M, int64_t K) { return M == 1 || (M ==
 inline bool swap_beats_gemv(int64_t M, int64_t N, int64_t K) {
   return (M >= 5 && N >= 6144) || (M >= 4 && N >= 16384) || (M >= 9 && K >= 8192);
 }
-// Without the GEMV (K too deep for its shared-memory rows), the tensor-core
-// variant still beats one row block of the GEMM on wide or deep weights.
-constexpr int64_t kSwapAutoMaxM = 16;
-constexpr int64_t kSwapAutoMinN = 6144;
-constexpr int64_t kSwapAutoMinK = 8192;
+// Without the GEMV (K too deep for its shared-memory rows, or more than 16
+// rows), the tensor-core variant still beats one row block of the GEMM on wide
+// or deep weights: to 16 rows from 6144 wide or 8192 deep; to 20 rows from
+// 9216 wide (17 rows: 13.6 vs 14.4 us at 9216 x 3072, 13.8 vs 16.4 at
+// 12288 x 3072, 16.3 vs 17.7 at 18432 x 3072; even at 24 rows, behind from
+// 32); to 32 rows from 8192 deep (4096 x 8192: 16.4-19.2 vs 21.7-22.2 us;
+// 3072 x 12288: 27.2-29.7 vs 30.2-30.3; behind at 48 rows).
+inline bool swap_beats_gemm(int64_t M, int64_t N, int64_t K) {
+  return (M <= 16 && (N >= 6144 || K >= 8192)) || (M <= 20 && N >= 9216) ||
+         (M <= 32 && K >= 8192);
+}
 
 inline int swap_mpad(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
 
@@ -155,7 +161,7 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
   if (v == W8A8_VARIANT_AUTO) {
     if (gemv_fits(M, K, max_smem) && !swap_beats_gemv(M, N, K)) {
       v = W8A8_VARIANT_GEMV;
-    } else if (M <= kSwapAutoMaxM && (N >= kSwapAutoMinN || K >= kSwapAutoMinK)) {
+    } else if (swap_beats_gemm(M, N, K)) {
       // a handful of rows against a wide or deep weight: the tensor-core
       // small-M variant (its K shared among the CTAs of a cluster) streams
       // the weight faster than the GEMV's dot products or one row block of
