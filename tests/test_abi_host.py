@@ -323,7 +323,7 @@ def test_selector_plans_are_valid_for_random_shapes(M, n8, k16):
         assert 4 <= M <= 32
         assert ((M <= 16 and (N >= 6144 or K >= 8192)) or (M <= 20 and N >= 9216)
                 or K >= 8192)
-        assert tm == 128 and tn == 16 and tiles == _cdiv(N, 128)
+        assert tm == 128 and tn == (16 if M <= 16 else 32) and tiles == _cdiv(N, 128)
         ks = p["k_split"]
         assert 1 <= ks <= 8 and ks <= _cdiv(K, 128) and p["grid"] == tiles * ks
         return
