@@ -177,6 +177,16 @@ W8A8_API int w8a8_quant_act(const void *x_bf16, int64_t M, int64_t K, int64_t ld
 W8A8_API int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes);
 
 /*
+ * As w8a8_workspace_size, for the plan of a given variant (w8a8_variant;
+ * AUTO gives w8a8_workspace_size's answer): a caller that forces the pair
+ * kernel through w8a8_linear_ex sizes its workspace here, so that the K-split
+ * region of that plan fits (the automatic plan may have none).  Returns
+ * W8A8_ERR_UNSUPPORTED_SHAPE where the variant cannot run (M, N, K).
+ */
+W8A8_API int w8a8_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant,
+                                    size_t *bytes);
+
+/*
  * int8 GEMM + fused epilogue on already-quantized activations.
  * q int8 [M,K] dense, s_a fp32 [M], Wq int8 [N,K] dense, s_w fp32 [N],
  * bias bf16 [N] or NULL -> y bf16 [M,N] (row stride ldy).
@@ -199,7 +209,8 @@ W8A8_API int w8a8_linear(const int8_t *q, const float *s_a, int64_t M, int64_t K
 
 /* w8a8_linear with an explicit kernel variant (AUTO = the selector's choice).
  * GEMV requires M <= 16.  workspace as in w8a8_linear (GEMM_PAIR uses it for
- * the K-split tail when large enough; NULL runs the pair kernel unsplit). */
+ * the K-split tail when it holds w8a8_workspace_size_ex(M, N, K,
+ * W8A8_VARIANT_GEMM_PAIR) bytes; NULL runs the pair kernel unsplit). */
 W8A8_API int w8a8_linear_ex(const int8_t *q, const float *s_a, int64_t M, int64_t K,
                    const int8_t *Wq, const float *s_w, const void *bias_bf16_or_null, int64_t N,
                    void *y_bf16, int64_t ldy, int32_t *acc_debug_or_null,

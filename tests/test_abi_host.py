@@ -191,7 +191,7 @@ def _pair_items(tiles, split_tiles, per, kb, pairs, pair, nsplit=0):
 SPLIT_SHAPES = [(4352, 9216, 3072), (4352, 12288, 3072), (4352, 3072, 12288), (512, 1024, 12288),
                 (640, 768, 1024), (200, 136, 12288), (1280, 4096, 1024), (2560, 8192, 512),
                 (8704, 9216, 3072), (16384, 3072, 12288), (512, 9472, 3072), (8704, 3072, 12288),
-                (600, 2056, 12288), (768, 1024, 133120)]
+                (600, 2056, 12288), (768, 1024, 133120), (2, 8, 133120)]
 
 
 @pytest.mark.parametrize("M,N,K", SPLIT_SHAPES)
@@ -261,6 +261,40 @@ def test_pair_k_split_plans():
     # the workspace covers the K-split region: counters + (split + pairs - 1) slots of 256 KiB
     n = w8a8.workspace_size(8704, 3072, 12288)
     assert n >= 8704 * 12288 + 4 * 8704 + (112 + 73) * 256 * 1024
+    # a forced pair plan gets its own K-split region even where the automatic
+    # plan (one round of 128 x 128 tiles here) has none
+    auto = w8a8.workspace_size(512, 1024, 12288)
+    assert w8a8.workspace_size(512, 1024, 12288, B.VARIANT_GEMM_PAIR) >= auto + (8 + 73) * 256 * 1024
+    assert w8a8.workspace_size(512, 1024, 12288, B.VARIANT_AUTO) == auto
+    assert w8a8.workspace_size(512, 1024, 12288, B.VARIANT_GEMM_BN256) == auto
+    with pytest.raises(w8a8.W8A8Error):
+        w8a8.workspace_size(17, 64, 256, B.VARIANT_GEMV_TC + 1)
+
+
+def test_selector_tile_width_and_pairs_follow_the_measured_rounds():
+    # 128-wide tiles only where they fill the rounds 1.4x better than 256-wide
+    # ones: 768 x 9216 x 3072 takes 3 rounds of 128-wide tiles, 2 of 256-wide
+    # ones or 1.5 of pairs (measured 29.5 / 25.3 / 24.1 us)
+    assert w8a8.select(768, 9216, 3072)["variant_name"] == "gemm_pair"
+    assert w8a8.select(384, 9216, 3072)["variant_name"] == "gemm_bn256"
+    assert w8a8.select(256, 9216, 3072)["variant_name"] == "gemm_bn128"   # one round either way
+    assert w8a8.select(768, 3072, 3072)["variant_name"] == "gemm_bn128"
+    # pairs from 256 rows when they fill the rounds as well (300 x 18432: 144
+    # pair tiles, 26.4 us against 26.6 for 256-wide tiles, 29.4 for 128-wide)
+    assert w8a8.select(300, 18432, 3072)["variant_name"] == "gemm_pair"
+    # under one round of pair tiles that one round of single-CTA tiles holds:
+    # the single-CTA tiles at K = 3072 (512 x 9216: 18.0 vs 18.9 us) and where
+    # the pair plan would share K out (1024 x 3072 x 12288: 47.9 vs 51.7) ...
+    assert w8a8.select(512, 9216, 3072)["variant_name"] == "gemm_bn256"
+    assert w8a8.select(1024, 3072, 12288)["variant_name"] == "gemm_bn256"
+    assert w8a8.select(1024, 3072, 12288, variant=B.VARIANT_GEMM_PAIR)["split_tiles"] == 48
+    # ... the pairs, unsplit, on deep K (512 x 9216 x 12288: 47.1 vs 52.0)
+    p = w8a8.select(512, 9216, 12288)
+    assert p["variant_name"] == "gemm_pair" and p["split_tiles"] == 0 and p["num_tiles"] == 72
+    # the full-size layers keep the pair kernel
+    for M, N, K in ((4352, 9216, 3072), (4352, 3072, 12288), (8704, 3072, 3072),
+                    (8704, 24576, 3072), (16384, 3072, 12288)):
+        assert w8a8.select(M, N, K)["variant_name"] == "gemm_pair", (M, N, K)
 
 
 def test_selector_at_17_rows_follows_the_measured_crossovers():

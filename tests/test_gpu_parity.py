@@ -591,6 +591,9 @@ def test_pair_k_split_matches_unsplit_and_oracle(M, N, K):
     accumulators and y, in full -- and against the oracle on sampled rows."""
     plan = w8a8.select(M, N, K, variant=B.VARIANT_GEMM_PAIR)
     assert plan["split_tiles"] > 0
+    # the binding sizes the workspace for the forced plan, K-split region included
+    assert w8a8.workspace_size(M, N, K, B.VARIANT_GEMM_PAIR) >= M * K + 4 * M + 16 * 4096 * 4 * (
+        plan["split_tiles"] + plan["grid"] // 2 - 1)
     rng = np.random.default_rng(M + N + K)
     q = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
     wq = rng.integers(-127, 128, size=(N, K), dtype=np.int8)
@@ -622,7 +625,8 @@ def test_pair_k_split_repeated_calls_on_one_workspace():
     wq = rng.integers(-127, 128, size=(N, K), dtype=np.int8)
     Wq = torch.from_numpy(wq).cuda()
     ones_n = torch.ones(N, device="cuda")
-    ws = torch.empty((w8a8.workspace_size(M, N, K),), dtype=torch.uint8, device="cuda")
+    ws = torch.empty((w8a8.workspace_size(M, N, K, B.VARIANT_GEMM_PAIR),), dtype=torch.uint8,
+                     device="cuda")
     qs = [rng.integers(-127, 128, size=(M, K), dtype=np.int8) for _ in range(3)]
     accs = [w8a8.linear(torch.from_numpy(q).cuda(), torch.ones(M, device="cuda"), Wq, ones_n,
                         acc_debug=True, variant=B.VARIANT_GEMM_PAIR, workspace=ws) for q in qs]
@@ -647,7 +651,8 @@ def test_pair_k_split_ignores_counter_words_planted_with_the_live_tag():
     args = (torch.from_numpy(q).cuda(), torch.ones(M, device="cuda"), torch.from_numpy(wq).cuda(),
             torch.ones(N, device="cuda"))
     ref_plain = w8a8.linear(*args, acc_debug=True, variant=B.VARIANT_GEMM_PAIR, split=False)
-    ws = torch.empty((w8a8.workspace_size(M, N, K),), dtype=torch.uint8, device="cuda")
+    ws = torch.empty((w8a8.workspace_size(M, N, K, B.VARIANT_GEMM_PAIR),), dtype=torch.uint8,
+                     device="cuda")
     for _ in range(2):
         torch.cuda.synchronize()
         word = np.array([(B.debug_peek_tag() << 8) | 3], dtype=np.uint64).view(np.int64)[0]
@@ -758,9 +763,9 @@ def _fused_call(x, Wq, s_w, b, y, ws, ws_bytes, q_out=None, s_a_out=None, option
 # (8704 x 3072 x 3072, the first round's rows through the ring, the rest
 # interleaved with epilogues), a ragged 12288-wide K with two bulk rows per
 # warp, and K = 6144 (two rows in flight per warp's share of the ring).
-FUSED_CASES = [(4352, 9216, 3072, 3072), (1091, 3072, 3072, 3072), (1537, 2048, 3072, 3200),
-               (2048, 2048, 512, 512), (4352, 3072, 12288, 12288), (8704, 3072, 3072, 3072),
-               (2600, 1024, 12288, 12296), (3000, 4096, 6144, 6144)]
+FUSED_CASES = [(4352, 9216, 3072, 3072), (1091, 6144, 3072, 3072), (1537, 4096, 3072, 3200),
+               (2048, 4096, 512, 512), (4352, 3072, 12288, 12288), (8704, 3072, 3072, 3072),
+               (2600, 2048, 12288, 12296), (3000, 4096, 6144, 6144)]
 
 
 @pytest.mark.parametrize("M,N,K,ldx", FUSED_CASES)
@@ -804,7 +809,9 @@ def test_quantization_fused_into_pair_launch_replayed_in_a_cuda_graph():
     """The one-launch layer captured in a CUDA graph (its row-block counters
     are cleared by a memset node of the same graph) and replayed on new
     activations each time: every replay must equal the oracle."""
-    M, N, K = 2304, 2048, 3072
+    M, N, K = 2304, 4096, 3072
+    plan = w8a8.select(M, N, K)
+    assert plan["variant_name"] == "gemm_pair" and plan["quant_in_gemm_launch"] == 1
     w = synth.make_w(N, K, 23)
     wq, sw = oracle.quantize_weights(w)
     b = synth.make_bias(N, 23)

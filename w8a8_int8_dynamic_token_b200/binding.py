@@ -73,6 +73,7 @@ _SIGNATURES = {
     "w8a8_quant_act": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp], _int),
     "w8a8_unpack_int32_weights": ([_vp, _i64, _i64, _vp, _vp], _int),
     "w8a8_workspace_size": ([_i64, _i64, _i64, ctypes.POINTER(_sz)], _int),
+    "w8a8_workspace_size_ex": ([_i64, _i64, _i64, _int, ctypes.POINTER(_sz)], _int),
     "w8a8_linear": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp],
                     _int),
     "w8a8_linear_ex": ([_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _int, _vp,
@@ -149,6 +150,12 @@ def w8a8_quant_act(x, M, K, ldx, q, s_a, stream) -> int:
 def w8a8_workspace_size(M, N, K) -> tuple[int, int]:
     out = ctypes.c_size_t(0)
     st = lib().w8a8_workspace_size(M, N, K, ctypes.byref(out))
+    return st, int(out.value)
+
+
+def w8a8_workspace_size_ex(M, N, K, variant) -> tuple[int, int]:
+    out = ctypes.c_size_t(0)
+    st = lib().w8a8_workspace_size_ex(M, N, K, variant, ctypes.byref(out))
     return st, int(out.value)
 
 
@@ -295,9 +302,9 @@ def _switching(dev, stream):
 
 
 @functools.lru_cache(maxsize=1024)
-def workspace_size(M: int, N: int, K: int) -> int:
-    st, n = w8a8_workspace_size(M, N, K)
-    _check(st, "w8a8_workspace_size")
+def workspace_size(M: int, N: int, K: int, variant: int = VARIANT_AUTO) -> int:
+    st, n = w8a8_workspace_size_ex(M, N, K, variant)
+    _check(st, "w8a8_workspace_size_ex")
     return n
 
 
@@ -350,14 +357,14 @@ def quant_act(x: torch.Tensor, stream=None):
     return q, s_a
 
 
-def _workspace_for(M, N, K, workspace, dev):
+def _workspace_for(M, N, K, workspace, dev, variant=VARIANT_AUTO):
     """(tensor, pointer, bytes): the caller's workspace, or a fresh one of
-    workspace_size(M, N, K) bytes when `workspace` is None (allocated on the
-    launching stream, inside _launching).  The caller keeps the returned
+    workspace_size(M, N, K, variant) bytes when `workspace` is None (allocated
+    on the launching stream, inside _launching).  The caller keeps the returned
     tensor alive until the launch has been enqueued: the device memory must
     not return to the allocator before then, or an output allocated
     afterwards could share it."""
-    need = workspace_size(M, N, K)
+    need = workspace_size(M, N, K, variant)
     if workspace is None:
         if need == 0:
             return None, None, 0
@@ -393,7 +400,7 @@ def linear(q, s_a, Wq, s_w, bias=None, out=None, acc_debug=False, variant=VARIAN
     dev = _on_one_device(q=q, s_a=s_a, Wq=Wq, s_w=s_w, bias=bias,
                          out=None if acc_debug else out, workspace=workspace)
     with _launching(dev, stream) as s:
-        ws, ws_ptr, ws_bytes = (_workspace_for(M, N, K, workspace, dev) if split
+        ws, ws_ptr, ws_bytes = (_workspace_for(M, N, K, workspace, dev, variant) if split
                                 else (None, None, 0))
         if acc_debug:
             acc = torch.empty((M, N), dtype=torch.int32, device=dev)

@@ -154,6 +154,60 @@ inline int swap_max_split(int mpad) {
   }
 }
 
+// How the pair kernel runs its last round(s) of 256 x 256 tiles on `pairs`
+// CTA pairs: whole tiles in full rounds, then -- when it pays -- either the
+// last round's tiles cut along N into two 128-column tiles (nsplit = 2), or
+// the last one to two rounds' tiles shared out along K so that every pair gets
+// the same number of k-blocks (a problem of less than one round is shared out
+// entirely).  Every shared-out piece costs about two epilogues (its partial
+// sums written, or read back and added), some 24 k-blocks of MMA time, so
+// pieces are at least that long and the split must save at least that much
+// per pair on the tail.
+struct PairTail {
+  int64_t tile0;   // tiles run whole before the shared-out ones
+  int64_t per;     // k-blocks per pair of the shared-out tiles (0: none)
+  int64_t nsplit;  // 2: the last round's tiles cut along N
+};
+
+inline PairTail pair_tail(int64_t tiles, int64_t kb, int64_t pairs) {
+  PairTail t{tiles, 0, 1};
+  const int64_t full = tiles / pairs, rem = tiles % pairs;
+  if (full >= 1 && rem > 0 && 2 * rem <= pairs) {
+    // A last round of rem tiles on `pairs` pairs costs as much as a full
+    // round: cut each of its tiles along N into two 128-column tiles, one per
+    // pair.  (Narrow tiles read more operand bytes per MMA; at 64 columns the
+    // round becomes bandwidth-bound and gains nothing.)
+    t.nsplit = 2;
+    t.tile0 = full * pairs;
+  } else if (rem != 0) {
+    const int64_t t0 = full >= 1 ? (full - 1) * pairs : 0;
+    const int64_t units = (tiles - t0) * kb;
+    int64_t pp = cdiv(units, pairs);
+    if (pp < kSplitMinPiece) pp = kSplitMinPiece;
+    const int64_t tail_unsplit = (cdiv(tiles, pairs) - t0 / pairs) * kb;
+    if (tail_unsplit - pp >= kSplitMinGain && units <= INT32_MAX / 2) {
+      t.tile0 = t0;
+      t.per = pp;
+    }
+  }
+  return t;
+}
+
+// Tile width and pair selection for the GEMM, from whole-layer times on a
+// B200 (quantization included, CUDA graphs; 104 shapes of 48-8704 rows, N
+// 1024-18432, K 3072 and 12288).  Per round of 148 CTAs, 128-wide tiles take
+// 0.67-0.75x the time of 256-wide ones for half the work, so they must fill
+// the rounds 1.4x better to win (768 x 9216 x 3072: 29.5 us against 25.3 for
+// 256-wide tiles and 24.1 for pairs).  Pair tiles win from 256 rows where
+// they fill the rounds about as well -- except under one round of pair tiles
+// that one round of single-CTA tiles holds, where the pair kernel either
+// shares K out (1024 x 3072 x 12288: 51.7 us against 47.9) or, at K = 3072,
+// loses its fill and drain (512 x 9216 x 3072: 18.9 against 18.0); on deep K
+// unsplit pairs still win (512 x 9216 x 12288: 47.1 against 52.0).
+constexpr double kBn128MinFillGain = 1.4;
+constexpr int64_t kPairMinM = 256;
+constexpr int64_t kPairOneRoundMinK = 6144;
+
 int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int max_smem,
                 w8a8_plan *plan) {
   if (sms < 1) return W8A8_ERR_INVALID_ARG;
@@ -180,7 +234,7 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
                           (static_cast<double>(N) / (cdiv(N, 256) * 256));
       const double e128 = static_cast<double>(t128) / (cdiv(t128, sms) * sms) *
                           (static_cast<double>(N) / (cdiv(N, 128) * 128));
-      v = (e128 > 1.15 * e256) ? W8A8_VARIANT_GEMM_BN128 : W8A8_VARIANT_GEMM_BN256;
+      v = (e128 > kBn128MinFillGain * e256) ? W8A8_VARIANT_GEMM_BN128 : W8A8_VARIANT_GEMM_BN256;
       // CTA pairs (256 x 256 tiles) halve each CTA's operand traffic; use
       // them when the problem has enough rows that pair tiles fill the GPU
       // about as well as single-CTA tiles do.
@@ -191,7 +245,12 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
                         (static_cast<double>(N) / (cdiv(N, 256) * 256));
       const double e1 = (v == W8A8_VARIANT_GEMM_BN128 ? e128 : e256) *
                         (static_cast<double>(M) / (cdiv(M, kBM) * kBM));
-      if (M >= 512 && sms >= 2 && ep >= 0.95 * e1) v = W8A8_VARIANT_GEMM_PAIR;
+      const int64_t t1 = v == W8A8_VARIANT_GEMM_BN128 ? t128 : t256;
+      const bool one_round = pairs >= 1 && tp < pairs && t1 <= sms;
+      const bool pair_loses_one_round =
+          one_round && (K < kPairOneRoundMinK || pair_tail(tp, cdiv(K, kBK), pairs).per > 0);
+      if (M >= kPairMinM && sms >= 2 && ep >= 0.95 * e1 && !pair_loses_one_round)
+        v = W8A8_VARIANT_GEMM_PAIR;
     }
   }
   std::memset(plan, 0, sizeof(*plan));
@@ -233,33 +292,10 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     const int64_t tiles = cdiv(M, 256) * cdiv(N, 256);
     if (tiles > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
     const int64_t kb = cdiv(K, kBK);
-    // Whole tiles in full waves, then -- when it pays -- the last one to two
-    // waves' tiles shared out along K so that every pair gets the same number
-    // of k-blocks (a problem of less than one wave is shared out entirely).
-    // Every shared-out piece costs about two epilogues (its partial sums
-    // written, or read back and added), some 24 k-blocks of MMA time, so
-    // pieces are at least that long and the split must save at least that
-    // much per pair on the tail.
-    int64_t pairs = sms / 2, tile0 = tiles, per = 0, nsplit = 1;
-    const int64_t full = tiles / pairs, rem = tiles % pairs;
-    if (full >= 1 && rem > 0 && 2 * rem <= pairs) {
-      // A last round of rem tiles on `pairs` pairs costs as much as a full
-      // round: cut each of its tiles along N into two 128-column tiles, one
-      // per pair.  (Narrow tiles read more operand bytes per MMA; at 64
-      // columns the round becomes bandwidth-bound and gains nothing.)
-      nsplit = 2;
-      tile0 = full * pairs;
-    } else if (rem != 0) {
-      const int64_t t0 = full >= 1 ? (full - 1) * pairs : 0;
-      const int64_t units = (tiles - t0) * kb;
-      int64_t pp = cdiv(units, pairs);
-      if (pp < kSplitMinPiece) pp = kSplitMinPiece;
-      const int64_t tail_unsplit = (cdiv(tiles, pairs) - t0 / pairs) * kb;
-      if (tail_unsplit - pp >= kSplitMinGain && units <= INT32_MAX / 2) {
-        tile0 = t0;
-        per = pp;
-      }
-    }
+    int64_t pairs = sms / 2;
+    const int64_t full = tiles / pairs;
+    const PairTail tail = pair_tail(tiles, kb, pairs);
+    const int64_t tile0 = tail.tile0, per = tail.per, nsplit = tail.nsplit;
     if (tile0 == tiles && tiles < pairs) pairs = tiles;
     plan->tile_m = 256;
     plan->tile_n = 256;
@@ -1125,13 +1161,17 @@ int w8a8_select(int64_t M, int64_t N, int64_t K, int32_t num_sms, int variant,
 }
 
 int w8a8_workspace_size(int64_t M, int64_t N, int64_t K, size_t *bytes) {
+  return w8a8_workspace_size_ex(M, N, K, W8A8_VARIANT_AUTO, bytes);
+}
+
+int w8a8_workspace_size_ex(int64_t M, int64_t N, int64_t K, int variant, size_t *bytes) {
   if (!bytes) return W8A8_ERR_INVALID_ARG;
   int st = check_mk(M, K, K);
   if (st != W8A8_OK) return st;
   st = check_n(N, N);
   if (st != W8A8_OK) return st;
   w8a8_plan plan;
-  st = select_plan(M, N, K, 148, W8A8_VARIANT_AUTO, 232448, &plan);
+  st = select_plan(M, N, K, 148, variant, 232448, &plan);
   if (st != W8A8_OK) return st;
   *bytes = plan.variant == W8A8_VARIANT_GEMV && plan.quant_in_gemm_launch
                ? 0
