@@ -271,6 +271,23 @@ def test_pair_k_split_plans():
         w8a8.workspace_size(17, 64, 256, B.VARIANT_GEMV_TC + 1)
 
 
+def test_small_m_split_keeps_every_cluster_resident():
+    # clusters of s CTAs a 148-SM B200 holds at once (one CTA per SM), from
+    # the device's occupancy query for this kernel
+    held = {1: 148, 2: 74, 3: 45, 4: 33, 5: 26, 6: 22, 7: 15, 8: 15}
+    for N in range(128, 18433, 128):
+        for K in (256, 3072, 8192, 12288):
+            p = w8a8.select(16, N, K, variant=B.VARIANT_GEMV_TC)
+            tiles, s = p["num_tiles"], p["k_split"]
+            assert tiles <= held[s] or s == 1, (N, K, s)
+            assert tiles * s <= 148 or s == 1
+    # measured best split per tile count (M = 16): 24 tiles of 3072 x 12288 in
+    # fours (12.9 us; clusters of 6, of which only 22 fit: 20.1 us), 48 tiles
+    # in twos (9.2 us; threes: 13.7), 16 tiles in sixes, 8 in eights
+    for N, want in ((3072, 4), (6144, 2), (2048, 6), (1024, 8), (9216, 2), (18432, 1)):
+        assert w8a8.select(16, N, 12288, variant=B.VARIANT_GEMV_TC)["k_split"] == want, N
+
+
 def test_selector_tile_width_and_pairs_follow_the_measured_rounds():
     # 128-wide tiles only where they fill the rounds 1.4x better than 256-wide
     # ones: 768 x 9216 x 3072 takes 3 rounds of 128-wide tiles, 2 of 256-wide

@@ -232,12 +232,13 @@ def test_gemv_fused_and_unfused(M, N, K):
 
 
 # (M, N, K): activation rows padded to 16 / 32 / 64 / 128; one tile
-# (128 x 256, K shared by up to 8 CTAs), ragged N (1032), K not a multiple of
-# 128 (2064), the AdaLN shape (144 tiles, no split), the QKV weight (72 tiles,
-# K in two halves) and N = 3072 (24 tiles, K in six parts).
+# (128 x 256, K shared by up to 8 CTAs), ragged N (1032, K in eight parts), K
+# not a multiple of 128 (2064), the AdaLN shape (144 tiles, no split), the QKV
+# weight (72 tiles, K in two halves), N = 3072 (24 tiles, K in four parts),
+# 16 tiles with K in six parts, 14 tiles with K in seven, and 3 tiles in five.
 GEMV_TC_CASES = [(1, 128, 256), (2, 18432, 3072), (5, 1032, 2064), (16, 9216, 3072),
                  (17, 3072, 3072), (31, 3072, 12288), (64, 264, 3072), (100, 9216, 3072),
-                 (128, 1032, 12288), (3, 128, 16)]
+                 (128, 1032, 12288), (3, 128, 16), (16, 2048, 8192), (8, 1792, 4096)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMV_TC_CASES)

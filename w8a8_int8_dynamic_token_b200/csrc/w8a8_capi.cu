@@ -154,6 +154,34 @@ inline int swap_max_split(int mpad) {
   }
 }
 
+// Clusters of s CTAs (one CTA per SM) that a 148-SM B200 holds at once, as
+// CTAs: a cluster must fit within one GPC, so sizes that do not divide the
+// GPCs' SM counts leave SMs idle (cudaOccupancyMaxActiveClusters for the
+// small-M kernel: 148, 148, 135, 132, 130, 132, 105, 120 CTAs for s = 1..8).
+// Scaled to other SM counts.
+constexpr int kClusterCTAs148[9] = {0, 148, 148, 135, 132, 130, 132, 105, 120};
+inline int64_t max_active_clusters(int64_t s, int32_t sms) {
+  return static_cast<int64_t>(kClusterCTAs148[s]) * sms / 148 / s;
+}
+
+// CTAs per tile (the cluster size) of the small-M kernel: K shared among up
+// to 4 CTAs, or more while the grid stays within 2/3 of the SMs, and never
+// more clusters than fit at once (a second wave of clusters doubles the time:
+// 24 tiles of 3072 x 12288 at M = 16 took 20.1 us in clusters of 6, of which
+// 22 fit, against 12.9 us in clusters of 4).  Measured best per tile count at
+// M = 16-32: 8 tiles 4-8, 12 tiles 6, 16 tiles 4-6, 24 tiles 4, 32 tiles 3-4,
+// 48 tiles 2, 72 tiles 2, 144 tiles 1.
+inline int64_t swap_split(int64_t tiles, int64_t kb, int mpad, int32_t sms) {
+  int64_t want = (2 * static_cast<int64_t>(sms) / 3) / tiles;
+  if (want < 4) want = 4;
+  int64_t split = sms / tiles;
+  if (split > want) split = want;
+  if (split > swap_max_split(mpad)) split = swap_max_split(mpad);
+  if (split > kb) split = kb;
+  while (split > 1 && tiles > max_active_clusters(split, sms)) --split;
+  return split < 1 ? 1 : split;
+}
+
 // How the pair kernel runs its last round(s) of 256 x 256 tiles on `pairs`
 // CTA pairs: whole tiles in full rounds, then -- when it pays -- either the
 // last round's tiles cut along N into two 128-column tiles (nsplit = 2), or
@@ -260,11 +288,7 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
     const int mpad = swap_mpad(M);
     const int64_t tiles = cdiv(N, kBM);
     const int64_t kb = cdiv(K, kBK);
-    // K shared among the CTAs of a cluster until the tiles fill the SMs
-    int64_t split = sms / tiles;
-    if (split > swap_max_split(mpad)) split = swap_max_split(mpad);
-    if (split > kb) split = kb;
-    if (split < 1) split = 1;
+    const int64_t split = swap_split(tiles, kb, mpad, sms);
     if (tiles * split > INT32_MAX) return W8A8_ERR_UNSUPPORTED_SHAPE;
     plan->tile_m = kBM;
     plan->tile_n = mpad;
