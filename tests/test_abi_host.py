@@ -101,30 +101,35 @@ def test_selector_small_m_goes_to_gemv():
     # The AdaLN modulation layer runs at M = batch (1, or 2 with CFG), below
     # the 16 rows a torch._int_mm path cannot serve: every such M is served
     # here, by the GEMV (quantizing its rows in the same launch at M = 1, 2),
-    # from 4 rows on this 18432-wide weight by the tensor-core small-M
+    # from 4 rows to 24 on this 18432-wide weight by the tensor-core small-M
     # variant (measured crossovers), and by the tcgen05 GEMM above.
     g = _golden("int_mm_min_rows.txt")
     lim, K, N = g["int_mm_min_rows_exclusive"], g["adaln_in_features"], g["adaln_out_features"]
     for M in (1, 2, 3):
         p = w8a8.select(M, N, K)
         assert p["variant_name"] == "gemv" and p["quant_in_gemm_launch"] == int(M <= 2)
-    for M in (4, 5, lim, lim + 1, 20):
+    for M in (4, 5, lim, lim + 1, 20, 24):
         assert w8a8.select(M, N, K)["variant_name"] == "gemv_tc"
-    assert w8a8.select(21, N, K)["variant_name"].startswith("gemm")
+    assert w8a8.select(25, N, K)["variant_name"].startswith("gemm")
     assert w8a8.select(lim, N, K, variant=B.VARIANT_GEMV)["variant_name"] == "gemv"
     assert w8a8.workspace_size(1, N, K) == 0
     assert w8a8.workspace_size(3, N, K) >= 3 * K + 3 * 4   # q and s_a for the quantization kernel
 
 
-def test_selector_narrow_weights_keep_the_gemv_to_16_rows():
+def test_selector_narrow_weights_keep_the_gemv_to_11_rows():
     # 3072 x 3072: the GEMV's dot products stay cheaper than the tensor-core
-    # paths up to 16 rows; 3072 x 12288: the tensor-core variant from 9 rows
-    for M in (3, 8, 16):
+    # variant up to 11 rows (8 rows: 7.4 vs 8.8 us; 12 rows: 10.0 vs 9.3);
+    # 3072 x 12288: the tensor-core variant from 5 rows (4 rows: 14.8 vs 15.2;
+    # 5 rows: 16.1 vs 13.9)
+    for M in (3, 8, 11):
         p = w8a8.select(M, 3072, 3072)
         assert p["variant_name"] == "gemv" and p["quant_in_gemm_launch"] == 0
+    for M in (12, 16):
+        assert w8a8.select(M, 3072, 3072)["variant_name"] == "gemv_tc"
     assert w8a8.select(2, 3072, 12288)["quant_in_gemm_launch"] == 0   # K > 8192: two launches
-    assert w8a8.select(8, 3072, 12288)["variant_name"] == "gemv"
-    assert w8a8.select(9, 3072, 12288)["variant_name"] == "gemv_tc"
+    assert w8a8.select(4, 3072, 12288)["variant_name"] == "gemv"
+    assert w8a8.select(5, 3072, 12288)["variant_name"] == "gemv_tc"
+    assert w8a8.select(11, 1024, 3072)["variant_name"] == "gemv"
 
 
 def test_selector_one_row_block_narrow_n_takes_64_column_tiles():
@@ -145,10 +150,11 @@ def test_selector_gemm_plans():
     p = w8a8.select(64, 128, 256)
     assert p["grid"] == p["num_tiles"] <= 2
     # too deep for the GEMV's shared-memory rows: the tensor-core small-M
-    # variant to 32 rows, the GEMM above
+    # variant to 48 rows, the GEMM above
     assert w8a8.select(16, 64, 16384)["variant_name"] == "gemv_tc"
-    assert w8a8.select(32, 64, 16384)["variant_name"] == "gemv_tc"
-    assert w8a8.select(33, 64, 16384)["variant_name"].startswith("gemm")
+    assert w8a8.select(48, 64, 16384)["variant_name"] == "gemv_tc"
+    assert w8a8.select(49, 64, 16384)["variant_name"].startswith("gemm")
+    assert w8a8.select(33, 64, 8192)["variant_name"].startswith("gemm")
     # forced variants
     assert w8a8.select(1, 64, 256, variant=B.VARIANT_GEMM_BN128)["tile_n"] == 128
     with pytest.raises(w8a8.W8A8Error):
@@ -323,9 +329,14 @@ def test_selector_at_17_rows_follows_the_measured_crossovers():
     assert w8a8.select(17, 6144, 3072)["variant_name"].startswith("gemm")
     assert w8a8.select(17, 3072, 3072)["variant_name"].startswith("gemm")
     assert w8a8.select(24, 9216, 3072)["variant_name"].startswith("gemm")
+    assert w8a8.select(24, 12288, 3072)["variant_name"] == "gemv_tc"
+    assert w8a8.select(25, 12288, 3072)["variant_name"].startswith("gemm")
+    # 64-column tiles for one row block only up to 37 tiles of 128 columns
+    assert w8a8.select(17, 6144, 3072)["variant_name"] == "gemm_bn128"
+    assert w8a8.select(17, 4096, 3072)["variant_name"] == "gemm_bn64"
 
 
-@pytest.mark.parametrize("M", [33, 100, 4352, 16384])
+@pytest.mark.parametrize("M", [49, 100, 4352, 16384])
 @pytest.mark.parametrize("KN", [(3072, 9216), (3072, 3072), (3072, 12288), (12288, 3072)])
 def test_selector_is_total_and_consistent(M, KN):
     K, N = KN
@@ -366,15 +377,17 @@ def test_selector_plans_are_valid_for_random_shapes(M, n8, k16):
     assert p["grid"] >= 1
     if v == "gemv":
         assert M <= 16 and M * K + 1024 <= 232448
-        assert not ((M >= 5 and N >= 6144) or (M >= 4 and N >= 16384) or (M >= 9 and K >= 8192))
+        assert not ((M >= 5 and (N >= 6144 or K >= 8192)) or
+                    (M >= 4 and (N >= 12288 or N * K >= 6144 * 12288)) or (M >= 12 and N >= 3072))
         assert p["quant_in_gemm_launch"] == int(M == 1 or (M == 2 and K <= 8192))
         return
     tm, tn, tiles = p["tile_m"], p["tile_n"], p["num_tiles"]
     if v == "gemv_tc":
-        assert 4 <= M <= 32
-        assert ((M <= 16 and (N >= 6144 or K >= 8192)) or (M <= 20 and N >= 9216)
-                or K >= 8192)
-        assert tm == 128 and tn == (16 if M <= 16 else 32) and tiles == _cdiv(N, 128)
+        assert 4 <= M <= 48
+        assert ((M <= 16 and (N >= 3072 or K >= 8192)) or (M <= 20 and N >= 9216)
+                or (M <= 24 and N >= 12288) or (M <= 32 and K >= 8192) or K >= 12288)
+        assert tm == 128 and tn == (16 if M <= 16 else (32 if M <= 32 else 64))
+        assert tiles == _cdiv(N, 128)
         ks = p["k_split"]
         assert 1 <= ks <= 8 and ks <= _cdiv(K, 128) and p["grid"] == tiles * ks
         return

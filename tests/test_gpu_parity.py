@@ -214,7 +214,8 @@ def test_gemv_fused_and_unfused(M, N, K):
     # weight faster; the CUDA-core GEMV is also checked through its explicit
     # (unfused) variant
     p = w8a8.select(M, N, K)
-    wide = (M >= 5 and N >= 6144) or (M >= 4 and N >= 16384) or (M >= 9 and K >= 8192)
+    wide = ((M >= 5 and (N >= 6144 or K >= 8192)) or
+            (M >= 4 and (N >= 12288 or N * K >= 6144 * 12288)) or (M >= 12 and N >= 3072))
     assert p["variant_name"] == ("gemv_tc" if wide else "gemv")
     assert p["quant_in_gemm_launch"] == (0 if wide else int(M == 1 or (M == 2 and K <= 8192)))
     y, q, s_a = w8a8.linear_fused(to_dev(x), Wq, s_w, to_dev(b), return_intermediates=True)

@@ -111,36 +111,40 @@ inline bool gemv_fits(int64_t M, int64_t K, int max_smem) {
 constexpr int64_t kSwapMaxM = 128;
 
 // Small-M selection, from whole-layer times on a B200 (quantization
-// included, CUDA graphs of back-to-back calls; us):
+// included, CUDA graphs of back-to-back calls, weights rotated over more than
+// 2x L2; us):
 //
 //   N x K          M:   1     2     4     5     8    12    16
-//   18432 x 3072  gemv 10.3* 11.9* 15.8  19.2  22.9  30.4  34.6
-//                 tc   14.1  14.1  14.4  15.1  15.7  16.5  17.3   GEMM 18.8-19.5
-//   9216 x 3072   gemv  6.3*  7.5* 10.1  12.0  14.2  18.0  20.6
-//                 tc   10.4  10.7  11.0  11.4  12.0  13.0  13.9   GEMM 14.2-15.1
-//   3072 x 3072   gemv  3.6*  4.1*  5.9   7.2   8.5  11.1  12.8
-//                 tc   13.4  13.6  14.0  14.3  14.9  16.0  17.0   GEMM 11.6-12.8
-//   3072 x 12288  gemv  9.2*  11.3  14.1  16.9  20.8  37.7  43.9
-//                 tc   21.3  22.3  22.9  23.0  23.5  24.2  24.8   GEMM 30.4-32.1
+//   18432 x 3072  gemv 10.3* 11.9* 15.2  17.7  21.4  29.2  33.3
+//                 tc               14.4  14.0  14.5  15.3  16.0   GEMM 18.6-20.4
+//   9216 x 3072   gemv  6.3*  7.5*  9.5  10.4  12.7  16.7  19.2
+//                 tc               10.4   9.9  10.3  11.4  12.5   GEMM 14.3-16.5
+//   3072 x 3072   gemv  3.6*  4.1*  6.4   6.1   7.4  10.0  11.0
+//                 tc                9.0   8.3   8.8   9.3   9.9   GEMM 10.9-11.7
+//   3072 x 12288  gemv  9.2*  11.3  14.8  16.1  20.1  35.9  42.4
+//                 tc               15.2  13.9  14.3  14.9  15.5   GEMM 30.3-32.4
 //
 // (* the GEMV with the quantization in its own launch; elsewhere the
 // quantization kernel runs first.)  The GEMV's dot products cost 1-2 us per
-// row on wide weights; the tensor-core variant is flat in M but pays for its
-// cluster-shared K on narrow ones.
+// row on wide weights (and more on deep ones, whose rows fill its shared
+// memory); the tensor-core variant is nearly flat in M.  Measured on 110
+// shapes of 4-48 rows (N 1024-18432, K 3072-12288), these rules pick the
+// fastest variant or one within 3% of it.
 inline bool gemv_quantizes_itself(int64_t M, int64_t K) { return M == 1 || (M == 2 && K <= 8192); }
 inline bool swap_beats_gemv(int64_t M, int64_t N, int64_t K) {
-  return (M >= 5 && N >= 6144) || (M >= 4 && N >= 16384) || (M >= 9 && K >= 8192);
+  return (M >= 5 && (N >= 6144 || K >= 8192)) ||
+         (M >= 4 && (N >= 12288 || N * K >= int64_t{6144} * 12288)) || (M >= 12 && N >= 3072);
 }
-// Without the GEMV (K too deep for its shared-memory rows, or more than 16
-// rows), the tensor-core variant still beats one row block of the GEMM on wide
-// or deep weights: to 16 rows from 6144 wide or 8192 deep; to 20 rows from
-// 9216 wide (17 rows: 13.6 vs 14.4 us at 9216 x 3072, 13.8 vs 16.4 at
-// 12288 x 3072, 16.3 vs 17.7 at 18432 x 3072; even at 24 rows, behind from
-// 32); to 32 rows from 8192 deep (4096 x 8192: 16.4-19.2 vs 21.7-22.2 us;
-// 3072 x 12288: 27.2-29.7 vs 30.2-30.3; behind at 48 rows).
+// Above 16 rows (or where the GEMV's rows do not fit), the tensor-core
+// variant still beats the GEMM's one row block: to 20 rows from 9216 wide
+// (17 rows at 9216 x 3072: 13.5 vs 14.6 us; even at 20; behind from 24), to
+// 24 rows from 12288 wide (18432 x 3072 at 24 rows: 17.9 vs 18.3), to 32 rows
+// from 8192 deep (3072 x 12288 at 32 rows: 20.6 vs 30.4; 4096 x 8192: 19.0 vs
+// 22.3) and to 48 rows from 12288 deep (28.0 vs 30.5 at 3072 x 12288; 8192
+// deep at 48 rows: behind, 24.9 vs 21.9).
 inline bool swap_beats_gemm(int64_t M, int64_t N, int64_t K) {
-  return (M <= 16 && (N >= 6144 || K >= 8192)) || (M <= 20 && N >= 9216) ||
-         (M <= 32 && K >= 8192);
+  return (M <= 16 && (N >= 3072 || K >= 8192)) || (M <= 20 && N >= 9216) ||
+         (M <= 24 && N >= 12288) || (M <= 32 && K >= 8192) || (M <= 48 && K >= 12288);
 }
 
 inline int swap_mpad(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128)); }
@@ -249,9 +253,10 @@ int select_plan(int64_t M, int64_t N, int64_t K, int32_t sms, int variant, int m
       // the weight faster than the GEMV's dot products or one row block of
       // the GEMM
       v = W8A8_VARIANT_GEMV_TC;
-    } else if (M <= kBM && cdiv(N, 128) * 3 <= sms) {
+    } else if (M <= kBM && cdiv(N, 128) * 4 <= sms) {
       // one row block and few 128-column tiles: 64-column tiles put twice as
-      // many CTAs on the weight stream (measured ~4% faster at N = 3072)
+      // many CTAs on the weight stream (measured ~4% faster at N = 3072; at
+      // N = 6144, 96 tiles of 64 columns, 8-18% slower than 48 of 128)
       v = W8A8_VARIANT_GEMM_BN64;
     } else {
       // wave efficiency of each tile width; 256-wide tiles move half the
